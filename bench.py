@@ -1,0 +1,344 @@
+"""Benchmark of one CD-RGE update (all probe losses, coefficients, update) on
+B200 through the C ABI.  Prints one JSON line on rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+
+A step is zo_probe_losses + zo_coeffs + zo_update over one synthetic batch of
+the named workload (default "overfit", the single-batch overfitting setting;
+also tiny, charlm, lstm270m, lstm1b).  `value` is CD-RGE steps/s of the whole
+job (device time, inputs resident in HBM, L2 flushed before every step and
+the flush not timed).  `e2e` is the same metric through zo_step_host with the
+step's tokens/targets copied from pinned host memory and L+/L- read back.
+With N > 1 (torchrun) every rank runs an independent replica on its own batch
+(weak scaling; no collective in the data path) and the time is the max over
+ranks.  `--impl reference` times the fp64 CPU oracle instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import workloads as W  # noqa: E402
+
+METRIC = "CD-RGE steps/s and perturbed-forward tokens/s on 1 B200; % of roofline"
+L2_BYTES = 126 * 1024 * 1024
+CLOCK_QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                "sm_max_mhz": d.get("sm_max_mhz", 1965.0), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "sm_max_mhz": 1965.0, "source": "fallback"}
+
+
+def fp32_alu_peak_tflops(sm_mhz):
+    """fp32 CUDA-core peak: 148 SMs x 128 FP32 lanes x 2 flops (FMA) x clock."""
+    return 148 * 128 * 2 * sm_mhz * 1e6 / 1e12
+
+
+def forward_macs_per_token(cfg):
+    m = cfg.vocab * cfg.hidden
+    for l in range(cfg.layers):
+        m += 4 * cfg.hidden * ((cfg.embed if l == 0 else cfg.hidden) + cfg.hidden)
+    return m
+
+
+def batches(cfg, n, rank):
+    """n (tokens, targets) batches for rank `rank`: fresh Markov batches per
+    step for the LM workloads, the fixed batch for copy / overfit."""
+    if cfg.task in ("copy", "overfit"):
+        b = W.batch_for(cfg)
+        return [b] * n
+    return [W.markov_batch(cfg.batch, cfg.seq, step=1000 * rank + k, vocab=cfg.vocab) for k in range(n)]
+
+
+class ClockSampler:
+    def __init__(self, gpu_index, path):
+        self.path = path
+        self.proc = None
+        try:
+            self.f = open(path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={gpu_index}", f"--query-gpu={CLOCK_QUERY}", "--format=csv,noheader",
+                 "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], [], set()
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1].split()[0]))
+                mx.append(float(f[2].split()[0]))
+            except ValueError:
+                continue
+            names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+            for nm, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def run_ours(args, cfg):
+    import torch
+    import torch.distributed as dist
+
+    import zero_order_recurrent_b200 as zo
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300))
+    zo.load_library()
+    dev = torch.device("cuda", local)
+    n, eps, eta = cfg.n_pert, cfg.eps, cfg.eta
+    theta_h = W.init_theta(cfg)
+    theta = torch.from_numpy(theta_h).to(dev)
+    del theta_h
+    K, Wm = args.steps, args.warmup
+    bl = batches(cfg, Wm + K, rank)
+    toks = [torch.from_numpy(t).to(dev) for t, _ in bl]
+    tgts = [torch.from_numpy(g).to(dev) for _, g in bl]
+    lp = torch.empty(n, device=dev)
+    lm = torch.empty(n, device=dev)
+    coef = torch.empty(n, device=dev)
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    ctx = zo.Context.for_config(cfg)
+    st = torch.cuda.current_stream()
+
+    def step(k):
+        zo.cdrge_step(ctx, theta, W.step_seed(k, run_seed=rank), n, eps, eta, toks[k], tgts[k],
+                      lp, lm, coef)
+
+    for k in range(Wm):
+        step(k)
+    torch.cuda.synchronize()
+    s = zo.zo_sync_status(ctx)
+    if s != zo.ZO_OK:
+        raise RuntimeError(f"warm-up failed: {zo.status_string(s)}")
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local, os.path.join(ROOT, "gpurun_out", f"clocks_rank{rank}.csv")) \
+        if os.path.isdir(os.path.join(ROOT, "gpurun_out")) or True else None
+    launches0 = zo.zo_kernel_launches()
+    zo.zo_profile(ctx, True)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    for k in range(K):
+        flush.fill_(float(k))                      # L2 flush, outside the timed window
+        ev[k][0].record(st)
+        step(Wm + k)
+        ev[k][1].record(st)
+    torch.cuda.synchronize()
+    zo.zo_profile(ctx, False)
+    launches = zo.zo_kernel_launches() - launches0
+    clocks = sampler.stop() if sampler else None
+    s = zo.zo_sync_status(ctx)
+    if s != zo.ZO_OK:
+        raise RuntimeError(f"timed steps failed: {zo.status_string(s)}")
+    ms = sum(a.elapsed_time(b) for a, b in ev)
+    kinds = {name: zo.zo_profile_read(ctx, kind) for name, kind in
+             (("cell", zo.ZO_KIND_CELL), ("loss", zo.ZO_KIND_LOSS), ("update", zo.ZO_KIND_UPDATE),
+              ("other", zo.ZO_KIND_OTHER))}
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+
+    # end-to-end through zo_step_host: pinned host inputs in, losses out
+    e2e = None
+    if not args.no_e2e:
+        ht = [torch.from_numpy(t).pin_memory() for t, _ in bl]
+        hg = [torch.from_numpy(g).pin_memory() for _, g in bl]
+        hp = torch.empty(n, dtype=torch.float32).pin_memory()
+        hm = torch.empty(n, dtype=torch.float32).pin_memory()
+        Ke = max(1, min(K, 5))
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        for k in range(Ke):
+            zo.zo_step_host(ctx, theta, W.step_seed(Wm + K + k, run_seed=rank), n, eps, eta, ht[k % len(ht)],
+                            hg[k % len(hg)], hp, hm)
+        torch.cuda.synchronize()
+        e_ms = (time.perf_counter() - t0) * 1e3
+        if world > 1:
+            t = torch.tensor([e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": world * Ke / (e_ms / 1e3), "unit": "steps/s",
+               "h2d_bytes_per_step": 2 * cfg.batch * cfg.seq * 4, "d2h_bytes_per_step": 2 * n * 4,
+               "steps": Ke}
+    ctx.close()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return {"ms": ms, "kinds": kinds, "clocks": clocks, "launches": launches, "e2e": e2e,
+            "rank": rank, "world": world}
+
+
+def roofline_for(cfg, kinds, clocks, pk):
+    n_cell, ms_cell, fl_cell, _ = kinds["cell"]
+    if cfg.dtype == "bf16":
+        achieved = fl_cell / (ms_cell / 1e3) / 1e12
+        peak = pk["bf16_tflops_sustained"]
+        return {"bound": "tensor", "kernel": "cell_tc_kernel (tcgen05 perturbed LSTM cell)",
+                "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+                "frac": round(achieved / peak, 4), "traffic": None,
+                "peak_source": f"{pk['source']} bf16 dense, sustained",
+                "launches": n_cell, "avg_launch_ms": round(ms_cell / max(n_cell, 1), 4)}
+    achieved = fl_cell / (ms_cell / 1e3) / 1e12
+    mhz = pk["sm_max_mhz"]
+    peak = fp32_alu_peak_tflops(mhz)
+    return {"bound": "alu", "kernel": "fp32_forward_kernel (persistent perturbed LSTM forward)",
+            "achieved": round(achieved, 3), "peak": round(peak, 2), "unit": "TFLOP/s",
+            "frac": round(achieved / peak, 4), "traffic": None,
+            "peak_source": f"fp32 FMA: 148 SMs x 128 lanes x 2 x {mhz:.0f} MHz",
+            "launches": n_cell, "avg_launch_ms": round(ms_cell / max(n_cell, 1), 4)}
+
+
+def oracle_sample(cfg, budget_s=15.0, rank=0):
+    """Time the fp64 oracle on a bounded sample of one step and extrapolate."""
+    import oracle as O
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        threads = 1
+    spec = (cfg.vocab, cfg.embed, cfg.hidden, cfg.layers)
+    theta = W.init_theta(cfg)
+    tok, tgt = batches(cfg, 1, rank)[0]
+    rows = None
+    if cfg.batch * cfg.seq * forward_macs_per_token(cfg) > 2e10:
+        rows = np.arange(min(cfg.batch, 32))
+    seed = W.step_seed(0)
+    t0 = time.perf_counter()
+    done = 0
+    while done < cfg.n_pert and (time.perf_counter() - t0) < budget_s:
+        O.probe_losses(theta, spec, seed, cfg.n_pert, cfg.eps, tok, tgt, probes=[done], rows=rows)
+        done += 1
+    t_fwd = time.perf_counter() - t0
+    rows_used = cfg.batch if rows is None else len(rows)
+    per_probe = t_fwd / done * (cfg.batch / rows_used)
+    # update cost on a slice of the parameters, scaled to the full vector
+    segs, d_pad = O.layout(*spec)
+    m = min(d_pad, 1 << 16)
+    idx = np.arange(m)
+    t1 = time.perf_counter()
+    O.update_at(theta, seed, min(cfg.n_pert, 8), np.zeros(min(cfg.n_pert, 8)), idx)
+    t_upd = (time.perf_counter() - t1) * (d_pad / m) * (cfg.n_pert / min(cfg.n_pert, 8))
+    step_s = per_probe * cfg.n_pert + t_upd
+    sample = (f"{done} of {cfg.n_pert} probes (both signs) over {rows_used} of {cfg.batch} rows, "
+              f"T={cfg.seq}, plus the update on {m} of {d_pad} parameters; extrapolated to one full step")
+    return {"value": 1.0 / step_s, "unit": "steps/s", "cores": threads, "kind": "oracle",
+            "sample": sample, "seconds": round(t_fwd + (time.perf_counter() - t1), 2)}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--config", default="overfit", choices=sorted(W.CONFIGS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    cfg = W.CONFIGS[args.config]
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    tokens_per_step = 2 * cfg.n_pert * cfg.batch * cfg.seq
+    config = {"workload": f"{cfg.name}: {cfg.layers}-layer LSTM V={cfg.vocab} E={cfg.embed} H={cfg.hidden}, "
+                          f"batch {cfg.batch} x seq {cfg.seq}, n_pert={cfg.n_pert}, eps=eta={cfg.eps}",
+              "params": int(W.segments(cfg.vocab, cfg.embed, cfg.hidden, cfg.layers)[1]),
+              "global_batch": cfg.batch * world, "seq_len": cfg.seq, "n_pert": cfg.n_pert,
+              "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+              "l2": "flushed (256 MB write) before every timed step, flush untimed",
+              "tokens": "seeded synthetic (workloads module)"}
+    dtype = "bf16" if cfg.dtype == "bf16" else "f32"
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        cb = oracle_sample(cfg, budget_s=max(5.0, 3.0 * args.steps))
+        v = cb["value"]
+        print(json.dumps({"metric": METRIC, "impl": "reference", "value": v, "unit": "steps/s",
+                          "perturbed_tokens_per_s": v * tokens_per_step, "n_gpus": world,
+                          "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 / v,
+                          "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                          "dtype": "f64", "data": "synthetic", "config": config,
+                          "cpu_baseline": cb,
+                          "e2e": {"value": v, "unit": "steps/s", "h2d_bytes_per_step": 0,
+                                  "d2h_bytes_per_step": 0}}), flush=True)
+        return
+
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    r = run_ours(args, cfg)
+    if rank != 0:
+        return
+    pk = peaks()
+    value = world * args.steps / (r["ms"] / 1e3)
+    out = {"metric": METRIC, "value": value, "unit": "steps/s",
+           "perturbed_tokens_per_s": value * tokens_per_step, "n_gpus": world, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": r["ms"] / args.steps, "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": dtype, "data": "synthetic",
+           "config": config, "roofline": roofline_for(cfg, r["kinds"], r["clocks"], pk)}
+    nu, msu, _, byu = r["kinds"]["update"]
+    if nu:
+        gbs = byu / (msu / 1e3) / 1e9
+        out["update_roofline"] = {"bound": "hbm", "achieved": round(gbs, 1), "peak": pk["hbm_gbs"],
+                                  "unit": "GB/s", "frac": round(gbs / pk["hbm_gbs"], 4),
+                                  "avg_launch_ms": round(msu / nu, 4)}
+    nl, msl, fll, byl = r["kinds"]["loss"]
+    if nl:
+        out["loss_kernel"] = {"launches": nl, "avg_launch_ms": round(msl / nl, 4),
+                              "tflops": round(fll / (msl / 1e3) / 1e12, 2),
+                              "gbs": round(byl / (msl / 1e3) / 1e9, 1)}
+    out["kernel_time_share"] = {k: round(v[1] / r["ms"], 4) for k, v in r["kinds"].items()}
+    out["e2e"] = r["e2e"]
+    out["gpu_launches"] = r["launches"]
+    out["clocks"] = r["clocks"]
+    if world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = oracle_sample(cfg)
+    print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

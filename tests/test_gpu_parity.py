@@ -1,0 +1,332 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on the
+same seeded inputs.  Tolerances: probe signs bit-exact; losses 1e-5 relative
+(fp32 path) and 1e-2 relative (bf16 path); update 1e-6 relative to
+|theta'| + sum|c|; sign(L+ - L-) agreement >= 95%; cos(g_gpu, g_oracle) >= 0.99."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import workloads as W
+import zero_order_recurrent_b200 as zo
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def library():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from zero_order_recurrent_b200 import build
+    build.build()
+    zo.load_library()
+
+
+def dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def spec_of(cfg):
+    return (cfg.vocab, cfg.embed, cfg.hidden, cfg.layers)
+
+
+def gpu_losses(ctx, theta, seed, n, eps, tok, tgt, rows=False):
+    B = tok.shape[0]
+    th = dev(theta)
+    lp = torch.empty(n, device="cuda")
+    lm = torch.empty(n, device="cuda")
+    rl = torch.empty(n * 2 * B, device="cuda") if rows else None
+    zo.zo_probe_losses(ctx, th, seed, n, eps, dev(tok), dev(tgt), lp, lm, row_loss=rl)
+    assert zo.zo_sync_status(ctx) == zo.ZO_OK
+    out = (lp.cpu().numpy().astype(np.float64), lm.cpu().numpy().astype(np.float64))
+    if rows:
+        out = out + (rl.cpu().numpy().reshape(n, 2, B).astype(np.float64),)
+    return out
+
+
+def sign_agreement(lp_a, lm_a, lp_b, lm_b):
+    return float(np.mean(np.sign(np.asarray(lp_a) - lm_a) == np.sign(np.asarray(lp_b) - lm_b)))
+
+
+def estimate_cosine(spec, seed, probes, lp_a, lm_a, lp_b, lm_b):
+    G = O.probe_gram(spec, seed, probes)
+    return O.gram_cosine(np.asarray(lp_a) - lm_a, np.asarray(lp_b) - lm_b, G)
+
+
+# ---------------------------------------------------------------------------
+# a1: probe signs
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("seed", [W.step_seed(0), 0, (1 << 64) - 1, 0x0123456789ABCDEF])
+@pytest.mark.parametrize("probe,q0", [(0, 0), (1, 1000), (511, 12345), (65535, (1 << 32) - 3),
+                                      ((1 << 31) - 1, 7)])
+def test_sign_words_bit_exact(seed, probe, q0):
+    n = 67
+    out = torch.zeros(4 * n, dtype=torch.int32, device="cuda")
+    zo.zo_sign_words(seed, probe, q0, n, out)
+    torch.cuda.synchronize()
+    got = out.cpu().numpy().view(np.uint32).reshape(n, 4)
+    want = O.sign_words(seed, probe, q0, n)
+    assert np.array_equal(got, want)
+
+
+# ---------------------------------------------------------------------------
+# a5 / a6: coefficients and update
+# ---------------------------------------------------------------------------
+def _check_update(cfg, n, theta, seed, coeffs, ctx, idx=None):
+    th = dev(theta)
+    c = dev(coeffs.astype(np.float32))
+    zo.zo_update(ctx, th, seed, n, c)
+    assert zo.zo_sync_status(ctx) == zo.ZO_OK
+    got = th.cpu().numpy().astype(np.float64)
+    c64 = coeffs.astype(np.float32).astype(np.float64)
+    if idx is None:
+        want = O.update(theta, spec_of(cfg), seed, n, c64)
+        tol = 1e-6 * (np.abs(want) + np.abs(c64).sum())
+        assert np.all(np.abs(got - want) <= tol)
+        mask = O.real_mask(*spec_of(cfg))
+        assert np.array_equal(got[~mask], theta[~mask])
+    else:
+        want = O.update_at(theta, seed, n, c64, idx)
+        tol = 1e-6 * (np.abs(want) + np.abs(c64).sum())
+        assert np.all(np.abs(got[idx] - want) <= tol)
+    return th
+
+
+@pytest.mark.parametrize("name,n", [("tiny", 8), ("overfit", 512), ("overfit", 37)])
+def test_update_matches_oracle(name, n):
+    cfg = W.CONFIGS[name]
+    theta = W.init_theta(cfg)
+    seed = W.step_seed(5)
+    coeffs = np.random.default_rng(n).standard_normal(n) * 1e-3
+    with zo.Context.for_config(cfg) as ctx:
+        _check_update(cfg, n, theta, seed, coeffs, ctx)
+
+
+def test_update_bf16_context_sampled_and_shadow():
+    """charlm-size theta: sampled indices against the oracle; the bf16 shadow
+    the update writes equals a fresh cast of theta' (losses bit-identical)."""
+    cfg = W.CONFIGS["charlm"]
+    theta = W.init_theta(cfg)
+    seed = W.step_seed(1)
+    n = cfg.n_pert
+    coeffs = np.random.default_rng(0).standard_normal(n) * 1e-4
+    rng = np.random.default_rng(1)
+    mask = O.real_mask(*spec_of(cfg))
+    idx = np.sort(rng.choice(np.nonzero(mask)[0], 20000, replace=False))
+    with zo.Context.for_config(cfg, max_batch=128, max_seq=2, chunk=2) as ctx:
+        th = _check_update(cfg, n, theta, seed, coeffs, ctx, idx)
+        tok, tgt = W.markov_batch(128, 2, step=3)
+        lp1 = torch.empty(2, device="cuda")
+        lm1 = torch.empty(2, device="cuda")
+        zo.zo_probe_losses(ctx, th, seed, 2, cfg.eps, dev(tok), dev(tgt), lp1, lm1)
+        zo.zo_invalidate_shadow(ctx)
+        lp2 = torch.empty(2, device="cuda")
+        lm2 = torch.empty(2, device="cuda")
+        zo.zo_probe_losses(ctx, th, seed, 2, cfg.eps, dev(tok), dev(tgt), lp2, lm2)
+        assert zo.zo_sync_status(ctx) == zo.ZO_OK
+        assert torch.equal(lp1, lp2) and torch.equal(lm1, lm2)
+
+
+def test_coefficients_match_formula():
+    n = 300
+    rng = np.random.default_rng(2)
+    lp = (2.3 + 1e-3 * rng.standard_normal(n)).astype(np.float32)
+    lm = (2.3 + 1e-3 * rng.standard_normal(n)).astype(np.float32)
+    with zo.Context(10, 16, 32, 1) as ctx:
+        out = torch.empty(n, device="cuda")
+        zo.zo_coeffs(ctx, dev(lp), dev(lm), n, 1e-3, 5e-4, out)
+        assert zo.zo_sync_status(ctx) == zo.ZO_OK
+        want = O.coefficients(lp, lm, n, 1e-3, 5e-4)
+        assert np.allclose(out.cpu().numpy(), want, rtol=1e-6, atol=0)
+
+
+# ---------------------------------------------------------------------------
+# a0-a4 on the fp32 path (tiny, overfit)
+# ---------------------------------------------------------------------------
+def test_fp32_tiny_full_step_matches_oracle():
+    cfg = W.CONFIGS["tiny"]
+    theta = W.init_theta(cfg)
+    tok, tgt = W.batch_for(cfg)
+    seed = W.step_seed(0)
+    with zo.Context.for_config(cfg) as ctx:
+        lp, lm = gpu_losses(ctx, theta, seed, cfg.n_pert, cfg.eps, tok, tgt)
+    olp, olm = O.probe_losses(theta, spec_of(cfg), seed, cfg.n_pert, cfg.eps, tok, tgt)
+    assert np.allclose(lp, olp, rtol=1e-5, atol=0)
+    assert np.allclose(lm, olm, rtol=1e-5, atol=0)
+    assert sign_agreement(lp, lm, olp, olm) >= 0.95
+    assert estimate_cosine(spec_of(cfg), seed, range(cfg.n_pert), lp, lm, olp, olm) >= 0.99
+
+
+def test_fp32_overfit_full_launch_sampled_probes():
+    """overfit config as benchmarked (512 probes, T = 100); the oracle checks a
+    sample of 24 probes spread over the range."""
+    cfg = W.CONFIGS["overfit"]
+    theta = W.init_theta(cfg)
+    tok, tgt = W.batch_for(cfg)
+    seed = W.step_seed(0)
+    with zo.Context.for_config(cfg) as ctx:
+        lp, lm = gpu_losses(ctx, theta, seed, cfg.n_pert, cfg.eps, tok, tgt)
+    probes = list(range(0, 512, 23)) + [511]
+    olp, olm = O.probe_losses(theta, spec_of(cfg), seed, cfg.n_pert, cfg.eps, tok, tgt, probes=probes)
+    assert np.allclose(lp[probes], olp, rtol=1e-5, atol=0)
+    assert np.allclose(lm[probes], olm, rtol=1e-5, atol=0)
+    assert sign_agreement(lp[probes], lm[probes], olp, olm) >= 0.95
+    assert estimate_cosine(spec_of(cfg), seed, probes, lp[probes], lm[probes], olp, olm) >= 0.99
+
+
+@pytest.mark.parametrize("V,E,H,L,B,T,n,chunk,frac", [
+    (7, 5, 6, 3, 5, 4, 3, 0, 0.3),      # three layers, odd widths
+    (13, 8, 24, 2, 9, 3, 7, 3, 0.5),    # ragged row blocks, several chunks
+    (11, 12, 40, 1, 1, 1, 1, 0, 0.0),   # T = 1, one probe
+    (9, 4, 8, 2, 3, 5, 2, 0, 1.0),      # nothing scored: loss 0
+])
+def test_fp32_edge_cases(V, E, H, L, B, T, n, chunk, frac):
+    cfg = W.small_config(vocab=V, embed=E, hidden=H, layers=L)
+    theta = W.init_theta(cfg, seed=3)
+    tok, tgt = W.random_batch(B, T, V, seed=4, ignore_frac=frac)
+    seed = W.step_seed(2)
+    with zo.Context(V, E, H, L, "f32", B, T, chunk) as ctx:
+        lp, lm, rows = gpu_losses(ctx, theta, seed, n, 1e-3, tok, tgt, rows=True)
+    olp, olm, orp, orm = O.probe_losses(theta, (V, E, H, L), seed, n, 1e-3, tok, tgt, return_rows=True)
+    assert np.allclose(lp, olp, rtol=1e-5, atol=1e-7)
+    assert np.allclose(lm, olm, rtol=1e-5, atol=1e-7)
+    assert np.allclose(rows[:, 0], orp, rtol=1e-5, atol=1e-6)
+    assert np.allclose(rows[:, 1], orm, rtol=1e-5, atol=1e-6)
+
+
+def test_deterministic_repeat():
+    cfg = W.CONFIGS["tiny"]
+    theta = W.init_theta(cfg)
+    tok, tgt = W.batch_for(cfg)
+    with zo.Context.for_config(cfg) as ctx:
+        a = gpu_losses(ctx, theta, 7, 8, cfg.eps, tok, tgt)
+        b = gpu_losses(ctx, theta, 7, 8, cfg.eps, tok, tgt)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+
+
+# ---------------------------------------------------------------------------
+# error reporting
+# ---------------------------------------------------------------------------
+def test_token_out_of_range_is_reported():
+    cfg = W.CONFIGS["tiny"]
+    tok, tgt = W.batch_for(cfg)
+    tok = tok.copy()
+    tok[3, 4] = 10
+    with zo.Context.for_config(cfg) as ctx:
+        th = dev(W.init_theta(cfg))
+        lp = torch.empty(2, device="cuda")
+        lm = torch.empty(2, device="cuda")
+        zo.zo_probe_losses(ctx, th, 1, 2, 1e-3, dev(tok), dev(tgt), lp, lm)
+        assert zo.zo_sync_status(ctx) == zo.ZO_ERR_BOUNDS
+        assert zo.zo_sync_status(ctx) == zo.ZO_OK   # cleared
+
+
+def test_nonfinite_loss_keeps_theta():
+    cfg = W.CONFIGS["tiny"]
+    theta = W.init_theta(cfg)
+    theta[5] = np.nan
+    tok, tgt = W.batch_for(cfg)
+    with zo.Context.for_config(cfg) as ctx:
+        th = dev(theta)
+        lp = torch.empty(3, device="cuda")
+        lm = torch.empty(3, device="cuda")
+        c = torch.empty(3, device="cuda")
+        zo.cdrge_step(ctx, th, 11, 3, 1e-3, 1e-3, dev(tok), dev(tgt), lp, lm, c)
+        assert zo.zo_sync_status(ctx) == zo.ZO_ERR_NONFINITE
+        got = th.cpu().numpy()
+        assert np.array_equal(np.isnan(got), np.isnan(theta))
+        assert np.array_equal(got[~np.isnan(theta)], theta[~np.isnan(theta)])
+
+
+def test_host_step_matches_device_step():
+    cfg = W.CONFIGS["tiny"]
+    theta = W.init_theta(cfg)
+    tok, tgt = W.batch_for(cfg)
+    seed = W.step_seed(4)
+    with zo.Context.for_config(cfg) as ctx:
+        a = dev(theta)
+        lp = torch.empty(8, device="cuda")
+        lm = torch.empty(8, device="cuda")
+        c = torch.empty(8, device="cuda")
+        zo.cdrge_step(ctx, a, seed, 8, cfg.eps, cfg.eta, dev(tok), dev(tgt), lp, lm, c)
+        b = dev(theta)
+        hp = np.zeros(8, np.float32)
+        hm = np.zeros(8, np.float32)
+        zo.zo_step_host(ctx, b, seed, 8, cfg.eps, cfg.eta, tok, tgt, hp, hm)
+        assert torch.equal(a, b)
+        assert np.array_equal(hp, lp.cpu().numpy()) and np.array_equal(hm, lm.cpu().numpy())
+
+
+# ---------------------------------------------------------------------------
+# bf16 tensor-core path
+# ---------------------------------------------------------------------------
+def _bf16(x):
+    """Round fp32 to bf16 (round to nearest even), returned as fp32."""
+    u = np.asarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    r = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16) << 16
+    return r.astype(np.uint32).view(np.float32)
+
+
+@pytest.mark.parametrize("B,E,H", [(200, 64, 64), (128, 128, 128), (300, 256, 1024)])
+def test_tc_cell_preactivation_matches_emulation(B, E, H):
+    """One tensor-core cell step (layer 0, t = 0) against an fp64 evaluation of
+    the same bf16 operands: x = bf16(E +- eps p), W = bf16(bf16(W) +- bf16(eps) p)."""
+    V, n = 50, 2
+    cfg = W.small_config(vocab=V, embed=E, hidden=H, layers=1, dtype="bf16")
+    theta = W.init_theta(cfg, seed=8)
+    tok, _ = W.random_batch(B, 1, V, seed=9)
+    seed = W.step_seed(6)
+    eps = np.float32(1e-3)
+    segs, _ = O.layout(V, E, H, 1)
+    offE, offW, offb = segs[0][3], segs[1][3], segs[2][3]
+    with zo.Context(V, E, H, 1, "bf16", B, 1, n) as ctx:
+        out = torch.full((2 * n, B, 4 * H), float("nan"), device="cuda")
+        zo.zo_debug_cell_preact(ctx, dev(theta), seed, 0, n, float(eps), dev(tok), out)
+        assert zo.zo_sync_status(ctx) == zo.ZO_OK
+        got = out.cpu().numpy()
+    Wt = theta[offW:offW + 4 * H * (E + H)].reshape(4 * H, E + H)[:, :E]
+    for i in range(n):
+        pE = O.probe_signs(seed, i, offE, V * E).reshape(V, E).astype(np.float32)
+        pW = O.probe_signs(seed, i, offW, 4 * H * (E + H)).reshape(4 * H, E + H)[:, :E].astype(np.float32)
+        pb = O.probe_signs(seed, i, offb, 4 * H).astype(np.float32)
+        for s, sg in ((0, 1.0), (1, -1.0)):
+            x = _bf16((theta[offE:offE + V * E].reshape(V, E) + np.float32(sg) * eps * pE)[tok[:, 0]])
+            Wp = _bf16(_bf16(Wt) + np.float32(sg) * _bf16(np.float32(eps)) * pW)
+            bias = (theta[offb:offb + 4 * H] + np.float32(sg) * eps * pb).astype(np.float64)
+            want = x.astype(np.float64) @ Wp.astype(np.float64).T + bias
+            g = got[2 * i + s]
+            err = np.abs(g - want)
+            assert np.all(err <= 1e-4 * (np.abs(x).astype(np.float64) @ np.abs(Wp).T + 1e-3)), \
+                (i, s, float(err.max()))
+
+
+@pytest.mark.parametrize("V,E,H,L,B,T,n", [(50, 64, 64, 2, 200, 4, 4), (50, 128, 256, 1, 128, 3, 3)])
+def test_bf16_small_matches_oracle(V, E, H, L, B, T, n):
+    cfg = W.small_config(vocab=V, embed=E, hidden=H, layers=L, dtype="bf16")
+    theta = W.init_theta(cfg, seed=1)
+    tok, tgt = W.markov_batch(B, T, step=0, vocab=V)
+    seed = W.step_seed(3)
+    with zo.Context(V, E, H, L, "bf16", B, T, n) as ctx:
+        lp, lm, rows = gpu_losses(ctx, theta, seed, n, 1e-3, tok, tgt, rows=True)
+    olp, olm, orp, orm = O.probe_losses(theta, (V, E, H, L), seed, n, 1e-3, tok, tgt, return_rows=True)
+    assert np.allclose(lp, olp, rtol=1e-2) and np.allclose(lm, olm, rtol=1e-2)
+    assert np.allclose(rows[:, 0], orp, rtol=1e-2, atol=1e-3)
+    assert np.allclose(rows[:, 1], orm, rtol=1e-2, atol=1e-3)
+
+
+def test_bf16_charlm_full_size_two_probes():
+    """charlm exactly as benchmarked (64 probes, batch 1024, T = 10); the oracle
+    evaluates probes 0 and 1 over the whole batch."""
+    cfg = W.CONFIGS["charlm"]
+    theta = W.init_theta(cfg)
+    tok, tgt = W.batch_for(cfg, step=0)
+    seed = W.step_seed(0)
+    with zo.Context.for_config(cfg) as ctx:
+        lp, lm = gpu_losses(ctx, theta, seed, cfg.n_pert, cfg.eps, tok, tgt)
+    probes = [0, 1]
+    olp, olm = O.probe_losses(theta, spec_of(cfg), seed, cfg.n_pert, cfg.eps, tok, tgt, probes=probes)
+    assert np.allclose(lp[probes], olp, rtol=1e-2) and np.allclose(lm[probes], olm, rtol=1e-2)
+    assert sign_agreement(lp[probes], lm[probes], olp, olm) >= 0.95
+    assert estimate_cosine(spec_of(cfg), seed, probes, lp[probes], lm[probes], olp, olm) >= 0.99

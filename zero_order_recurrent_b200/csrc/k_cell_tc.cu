@@ -1,0 +1,674 @@
+// Perturbed LSTM cell on the 5th-generation tensor cores (sm_100a).
+//
+// For every probe-sign ps = 2*ci + s of a chunk, layer l and step t:
+//   G[ps] = [x_t | h_{t-1}][ps] (W_l + (s ? -eps : eps) P_{probe})^T + (b_l +- eps p),
+//   c_t = sigma(f) c_{t-1} + sigma(i) tanh(g),  h_t = sigma(o) tanh(c_t),
+// i.e. one complete forward step at Theta +- eps p_i (pith.science review,
+// "What carries the argument"; alex-wiki "Method").  The perturbed operand is
+// never stored in HBM: the bf16 shadow tile of W_l arrives by TMA, four
+// generator warps add +-eps in place from the probe's Philox words, and
+// tcgen05.mma consumes it with fp32 accumulation in tensor memory.
+//
+// CTA tile: MT sub-tiles of 128 batch rows x BN gate rows (BN/4 hidden units,
+// the four gate blocks side by side so the epilogue sees i, f, g, o of a unit
+// together) x 64-deep K stages.  Warp roles (320 threads):
+//   warp 0      TMA producer (A activations, W_l tile as 4 gate boxes)
+//   warp 1      TMEM allocator and MMA issuer
+//   warps 2..5  perturbation: W tile += +-eps p in shared memory
+//   warps 6..9  epilogue: TMEM -> gates -> c, h (TMEM lane quadrant = warp % 4)
+// Every mbarrier wait is bounded: past ~2 s the CTA raises an abort flag, the
+// error word gets ZO_ERR_TIMEOUT, all roles leave their loops, and tensor
+// memory is freed before exit.  No multicast form of any copy is used.
+#include <cudaTypedefs.h>
+
+#include "zo_common.cuh"
+#include "zo_internal.h"
+
+namespace zo {
+
+constexpr int kTcThreads = 320;
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+struct CellArgs {
+  int K0;          // input width of the layer
+  int H;
+  int Ktot;        // K0 + H: row length of W_l
+  int nk;          // K stages to run (K0/64 at t == 0 where h_{-1} = 0)
+  int B, Bmax;
+  int m_tiles, n_tiles;
+  int64_t tiles;
+  int group;       // probe-sign x M tiles walked together (L2 locality)
+  uint64_t seed;
+  int probe0;
+  float eps;
+  int64_t offW;    // theta offset of W_l (Philox element index base)
+  const float* small_p;   // perturbed small segments
+  int64_t sstride, soffb; // per probe-sign stride, offset of b_l
+  float* cst;      // [P][Bmax][H] fp32
+  __nv_bfloat16* hout;    // [P][Bmax][H]
+  int first;       // t == 0: c_{-1} = 0
+  float* raw;      // optional [P][Bmax][4H] pre-activations (then c, h are not written)
+  unsigned* err;
+};
+
+// ---------------------------------------------------------------------------
+// PTX wrappers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t globaltimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Bounded wait.  Returns false (and raises the CTA abort flag) if the phase
+// did not complete within kWaitLimitNs, or if another role already aborted.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          unsigned* err) {
+  if (mbar_try(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try(bar, parity)) return true;
+    if ((i & 255) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer() - t0 > kWaitLimitNs) {
+        *abort_flag = 1;
+        latch(err, kErrTimeout);
+        return false;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int c0, int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1)
+      : "memory");
+}
+
+__device__ __forceinline__ void prefetch_map(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+__device__ __forceinline__ void fence_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// K-major operand tile in the 128-byte swizzled canonical layout: rows of
+// 64 bf16 (128 B), 8-row atoms of 1024 B; SBO = 1024 B, LBO unused (1),
+// descriptor version 1, layout type 2 (SWIZZLE_128B).
+__device__ __forceinline__ uint64_t umma_desc(uint32_t saddr) {
+  return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+// kind::f16 instruction descriptor: D fp32, A and B bf16, both K-major, M x N.
+__host__ __device__ constexpr uint32_t umma_idesc(int M, int N) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
+         ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   bar)
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+      "%12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_wait_ld() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ float tanh_fast(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float sigmoid_fast(float x) { return fmaf(0.5f, tanh_fast(0.5f * x), 0.5f); }
+
+__device__ __forceinline__ uint32_t bf16x2_add(uint32_t a, uint32_t b) {
+  __nv_bfloat162 r = __hadd2(*reinterpret_cast<__nv_bfloat162*>(&a),
+                             *reinterpret_cast<__nv_bfloat162*>(&b));
+  return *reinterpret_cast<uint32_t*>(&r);
+}
+
+// ---------------------------------------------------------------------------
+// Tile order: GA (probe-sign, M-tile) pairs walked together across all N tiles,
+// so a wave of CTAs shares a few A panels and a few W panels.
+// ---------------------------------------------------------------------------
+struct TileCoord {
+  int ps, m, n;
+};
+
+__device__ __forceinline__ TileCoord decode_tile(const CellArgs& a, int64_t tile, int P) {
+  const int64_t pm_count = (int64_t)P * a.m_tiles;
+  const int64_t per_group = (int64_t)a.group * a.n_tiles;
+  const int64_t g = tile / per_group;
+  const int64_t r = tile - g * per_group;
+  const int64_t first = g * a.group;
+  const int64_t ga = min((int64_t)a.group, pm_count - first);
+  const int64_t pm = first + r % ga;
+  TileCoord c;
+  c.n = (int)(r / ga);
+  c.ps = (int)(pm / a.m_tiles);
+  c.m = (int)(pm % a.m_tiles);
+  return c;
+}
+
+template <int MT, int BN, int STAGES, int ACC>
+struct TcCfg {
+  static constexpr int U = BN / 4;
+  static constexpr int A_SUB = 128 * 128;           // one 128-row sub-tile, bytes
+  static constexpr int A_BYTES = MT * A_SUB;
+  static constexpr int B_BYTES = BN * 128;
+  static constexpr int STAGE = A_BYTES + B_BYTES;
+  static constexpr int COLS = MT * BN;              // TMEM columns per accumulator
+  static constexpr int TMEM_COLS = COLS * ACC;
+  static constexpr int SMEM = STAGES * STAGE + 1024 + 256;
+  static_assert(BN % 64 == 0 && BN <= 256, "BN");
+  static_assert(TMEM_COLS == 128 || TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM columns");
+};
+
+template <int MT, int BN, int STAGES, int ACC>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    cell_tc_kernel(const __grid_constant__ CUtensorMap mapA0, const __grid_constant__ CUtensorMap mapA1,
+                   const __grid_constant__ CUtensorMap mapW, const CellArgs a, int P) {
+  using C = TcCfg<MT, BN, STAGES, ACC>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * C::STAGE);
+  // full[s], ready[s], empty[s], acc_full[ACC], acc_empty[ACC], drain
+  const uint32_t bar0 = smem_u32(bars);
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto ready_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (2 * STAGES + s); };
+  auto accf_bar = [&](int b) { return bar0 + 8u * (3 * STAGES + b); };
+  auto acce_bar = [&](int b) { return bar0 + 8u * (3 * STAGES + ACC + b); };
+  const uint32_t drain_bar = bar0 + 8u * (3 * STAGES + 2 * ACC);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * STAGES + 2 * ACC + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(ready_bar(s), 4);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int b = 0; b < ACC; ++b) {
+      mbar_init(accf_bar(b), 1);
+      mbar_init(acce_bar(b), 4);
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    fence_async_smem();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_map(&mapA0);
+    prefetch_map(&mapA1);
+    prefetch_map(&mapW);
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"(C::TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t it = 0;
+      bool ok = true;
+      for (int64_t tile = blockIdx.x; tile < a.tiles && ok; tile += gridDim.x) {
+        const TileCoord tc = decode_tile(a, tile, P);
+        const int row0 = tc.m * 128 * MT;
+        for (int kb = 0; kb < a.nk; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1;
+          if (!mbar_wait(empty_bar(s), ph ^ 1, abort_flag, a.err)) {
+            ok = false;
+            break;
+          }
+          mbar_expect_tx(full_bar(s), C::STAGE);
+          const uint32_t sa = sbase + s * C::STAGE;
+          const uint32_t sb = sa + C::A_BYTES;
+          const int kk = kb * 64;
+#pragma unroll
+          for (int mt = 0; mt < MT; ++mt) {
+            if (kk < a.K0)
+              tma_load_3d(sa + mt * C::A_SUB, &mapA0, full_bar(s), kk, row0 + mt * 128, tc.ps);
+            else
+              tma_load_3d(sa + mt * C::A_SUB, &mapA1, full_bar(s), kk - a.K0, row0 + mt * 128,
+                          tc.ps);
+          }
+#pragma unroll
+          for (int g = 0; g < 4; ++g)
+            tma_load_2d(sb + g * C::U * 128, &mapW, full_bar(s), kk, g * a.H + tc.n * C::U);
+        }
+      }
+      if (!ok) {
+        // let the copies already issued land before the CTA can exit
+        const uint32_t issued = it;
+        for (int s = 0; s < STAGES && (uint32_t)s < issued; ++s) {
+          const uint32_t n_iss = (issued - 1 - s) / STAGES + 1;
+          const uint64_t t0 = globaltimer();
+          while (!mbar_try(full_bar(s), (n_iss - 1) & 1) && globaltimer() - t0 < 100000000ull) {
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = umma_idesc(128, BN);
+      uint32_t it = 0, tcount = 0;
+      bool ok = true;
+      for (int64_t tile = blockIdx.x; tile < a.tiles && ok; tile += gridDim.x, ++tcount) {
+        const int ab = tcount % ACC;
+        const uint32_t aph = (tcount / ACC) & 1;
+        if (!mbar_wait(acce_bar(ab), aph ^ 1, abort_flag, a.err)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t dcol = tmem_base + ab * C::COLS;
+        for (int kb = 0; kb < a.nk; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1;
+          if (!mbar_wait(ready_bar(s), ph, abort_flag, a.err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = sbase + s * C::STAGE;
+          const uint64_t bdesc = umma_desc(sa + C::A_BYTES);
+#pragma unroll
+          for (int k16 = 0; k16 < 4; ++k16) {
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+              const uint64_t adesc = umma_desc(sa + mt * C::A_SUB);
+              umma_bf16(dcol + mt * BN, adesc + 2 * k16, bdesc + 2 * k16, idesc,
+                        (kb | k16) != 0 ? 1u : 0u);
+            }
+          }
+          umma_commit(empty_bar(s));
+        }
+        if (!ok) break;
+        umma_commit(accf_bar(ab));
+      }
+      // all MMAs issued by this thread complete before tensor memory is freed
+      umma_commit(drain_bar);
+      const uint64_t t0 = globaltimer();
+      while (!mbar_try(drain_bar, 0) && globaltimer() - t0 < 100000000ull) {
+      }
+    }
+  } else if (warp < 6) {
+    // ------------------------------------------------------------ perturbation
+    const int gt = threadIdx.x - 64;  // 0..127
+    constexpr int RPT = BN / 128 > 0 ? BN / 128 : 1;
+    const float epsf = a.eps;
+    const __nv_bfloat16 eb = __float2bfloat16_rn(epsf);
+    const uint32_t eps_bits = (uint32_t)(*reinterpret_cast<const uint16_t*>(&eb));
+    const uint32_t epsp2 = eps_bits | (eps_bits << 16);
+    const uint32_t epsn2 = epsp2 ^ 0x80008000u;
+    uint32_t it = 0;
+    bool ok = true;
+    for (int64_t tile = blockIdx.x; tile < a.tiles && ok; tile += gridDim.x) {
+      const TileCoord tc = decode_tile(a, tile, P);
+      const uint32_t probe = (uint32_t)(a.probe0 + (tc.ps >> 1));
+      const uint32_t e2 = (tc.ps & 1) ? epsn2 : epsp2;
+      int64_t cq[RPT];
+      uint4 cw[RPT];
+#pragma unroll
+      for (int rr = 0; rr < RPT; ++rr) cq[rr] = -1;
+      for (int kb = 0; kb < a.nk; ++kb, ++it) {
+        const int s = it % STAGES;
+        const uint32_t ph = (it / STAGES) & 1;
+        if (!mbar_wait(full_bar(s), ph, abort_flag, a.err)) {
+          ok = false;
+          break;
+        }
+        uint8_t* tileB = smem + s * C::STAGE + C::A_BYTES;
+#pragma unroll
+        for (int rr = 0; rr < RPT; ++rr) {
+          const int r = gt + rr * 128;
+          if (r < BN) {
+            const int g = r / C::U, u = r % C::U;
+            const int64_t R = (int64_t)g * a.H + (int64_t)tc.n * C::U + u;
+            const int64_t j0 = a.offW + R * a.Ktot + (int64_t)kb * 64;
+            const int64_t q = j0 >> 7;
+            if (q != cq[rr]) {
+              cw[rr] = sign_block(a.seed, probe, (uint64_t)q);
+              cq[rr] = q;
+            }
+            const bool upper = (j0 >> 6) & 1;
+            const uint32_t wlo = upper ? cw[rr].z : cw[rr].x;
+            const uint32_t whi = upper ? cw[rr].w : cw[rr].y;
+            uint8_t* row = tileB + r * 128;
+#pragma unroll
+            for (int c16 = 0; c16 < 8; ++c16) {
+              uint4* p = reinterpret_cast<uint4*>(row + ((c16 ^ (r & 7)) << 4));
+              uint4 v = *p;
+              const uint32_t w = (c16 < 4 ? wlo : whi) >> (4 * (c16 & 3));
+              v.x = bf16x2_add(v.x, ((w << 15) & 0x80008000u) ^ e2);
+              v.y = bf16x2_add(v.y, ((w << 14) & 0x80008000u) ^ e2);
+              v.z = bf16x2_add(v.z, ((w << 13) & 0x80008000u) ^ e2);
+              v.w = bf16x2_add(v.w, ((w << 12) & 0x80008000u) ^ e2);
+              *p = v;
+            }
+          }
+        }
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(ready_bar(s));
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int quad = warp & 3;
+    const int rloc = quad * 32 + lane;
+    uint32_t tcount = 0;
+    bool ok = true;
+    for (int64_t tile = blockIdx.x; tile < a.tiles && ok; tile += gridDim.x, ++tcount) {
+      const TileCoord tc = decode_tile(a, tile, P);
+      const int ab = tcount % ACC;
+      const uint32_t aph = (tcount / ACC) & 1;
+      if (!mbar_wait(accf_bar(ab), aph, abort_flag, a.err)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const float* bias = a.small_p + tc.ps * a.sstride + a.soffb;
+      for (int mt = 0; mt < MT; ++mt) {
+        const int b = tc.m * 128 * MT + mt * 128 + rloc;
+        const int64_t rowoff = ((int64_t)tc.ps * a.Bmax + b) * a.H;
+#pragma unroll 1
+        for (int u0 = 0; u0 < C::U; u0 += 16) {
+          uint32_t acc[4][16];
+#pragma unroll
+          for (int g = 0; g < 4; ++g)
+            tmem_ld16(tmem_base + ((uint32_t)(quad * 32) << 16) + ab * C::COLS + mt * BN +
+                          g * C::U + u0,
+                      acc[g]);
+          tmem_wait_ld();
+          if (b < a.B) {
+            const int unit0 = tc.n * C::U + u0;
+            float pre[4][16];
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+              const float4* bp = reinterpret_cast<const float4*>(bias + g * a.H + unit0);
+#pragma unroll
+              for (int q4 = 0; q4 < 4; ++q4) {
+                const float4 bv = __ldg(bp + q4);
+                pre[g][4 * q4 + 0] = __uint_as_float(acc[g][4 * q4 + 0]) + bv.x;
+                pre[g][4 * q4 + 1] = __uint_as_float(acc[g][4 * q4 + 1]) + bv.y;
+                pre[g][4 * q4 + 2] = __uint_as_float(acc[g][4 * q4 + 2]) + bv.z;
+                pre[g][4 * q4 + 3] = __uint_as_float(acc[g][4 * q4 + 3]) + bv.w;
+              }
+            }
+            if (a.raw) {
+              float* rp = a.raw + ((int64_t)tc.ps * a.Bmax + b) * 4 * a.H;
+#pragma unroll
+              for (int g = 0; g < 4; ++g)
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4)
+                  reinterpret_cast<float4*>(rp + g * a.H + unit0)[q4] =
+                      make_float4(pre[g][4 * q4], pre[g][4 * q4 + 1], pre[g][4 * q4 + 2],
+                                  pre[g][4 * q4 + 3]);
+            } else {
+              float cprev[16];
+              float4* cp = reinterpret_cast<float4*>(a.cst + rowoff + unit0);
+              if (a.first) {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) cprev[i] = 0.f;
+              } else {
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                  const float4 v = cp[q4];
+                  cprev[4 * q4] = v.x;
+                  cprev[4 * q4 + 1] = v.y;
+                  cprev[4 * q4 + 2] = v.z;
+                  cprev[4 * q4 + 3] = v.w;
+                }
+              }
+              float cn[16];
+              uint32_t hp[8];
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                const float ig = sigmoid_fast(pre[0][i]);
+                const float fg = sigmoid_fast(pre[1][i]);
+                const float gg = tanh_fast(pre[2][i]);
+                const float og = sigmoid_fast(pre[3][i]);
+                cn[i] = fmaf(fg, cprev[i], ig * gg);
+                const float hv = og * tanh_fast(cn[i]);
+                if (i & 1) {
+                  __nv_bfloat162 pr = __floats2bfloat162_rn(
+                      __uint_as_float(hp[i >> 1]), hv);
+                  hp[i >> 1] = *reinterpret_cast<uint32_t*>(&pr);
+                } else {
+                  hp[i >> 1] = __float_as_uint(hv);
+                }
+              }
+#pragma unroll
+              for (int q4 = 0; q4 < 4; ++q4)
+                cp[q4] = make_float4(cn[4 * q4], cn[4 * q4 + 1], cn[4 * q4 + 2], cn[4 * q4 + 3]);
+              uint4* hq = reinterpret_cast<uint4*>(a.hout + rowoff + unit0);
+              hq[0] = make_uint4(hp[0], hp[1], hp[2], hp[3]);
+              hq[1] = make_uint4(hp[4], hp[5], hp[6], hp[7]);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acce_bar(ab));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"(C::TMEM_COLS)
+                 : "memory");
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Host side: tensor maps and launch
+// ---------------------------------------------------------------------------
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// [P][B][K] bf16 activations, box 64 (K) x 128 (rows) x 1, 128-byte swizzle.
+bool map_act(CUtensorMap* m, void* base, int64_t K, int64_t B, int64_t P) {
+  auto enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)K, (cuuint64_t)B, (cuuint64_t)P};
+  cuuint64_t strides[2] = {(cuuint64_t)(K * 2), (cuuint64_t)(K * 2 * B)};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// W_l shadow [4H][Ktot] bf16, box 64 (K) x rows.
+bool map_w(CUtensorMap* m, void* base, int64_t Ktot, int64_t rows, int box_rows) {
+  auto enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)Ktot, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)(Ktot * 2)};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  cuuint32_t es[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Tile configuration.  Large K: 256 rows x 256 gate rows (all 512 TMEM
+// columns, epilogue not overlapped but amortised over K).  Small K: 128 x 256
+// with two accumulators so the epilogue of one tile overlaps the next.
+constexpr int kBN = 256;
+
+}  // namespace
+
+bool make_cell_maps(zo_ctx* c) {
+  const zo_model_spec& s = c->spec;
+  c->maps = new (std::nothrow) CellMaps();
+  if (!c->maps) return false;
+  const int64_t P = 2 * (int64_t)c->chunk, B = s.max_batch, E = s.embed, H = s.hidden;
+  const int L = s.layers;
+  bool ok = map_act(&c->maps->x, c->x, E, B, P);
+  for (int l = 0; l < L; ++l)
+    for (int par = 0; par < 2; ++par)
+      ok = ok && map_act(&c->maps->h[l][par], c->h + ((int64_t)l * 2 + par) * P * B * H, H, B, P);
+  for (int l = 0; l < L; ++l) {
+    const int64_t Ktot = (l == 0 ? E : H) + H;
+    ok = ok && map_w(&c->maps->w[l], c->shadow + c->seg.off[c->seg.W[l]], Ktot, 4 * H, kBN / 4);
+  }
+  return ok;
+}
+
+template <int MT, int BN, int STAGES, int ACC>
+static cudaError_t launch_cfg(const CUtensorMap& A0, const CUtensorMap& A1, const CUtensorMap& Wm,
+                              CellArgs a, int P, int sms, cudaStream_t st) {
+  using C = TcCfg<MT, BN, STAGES, ACC>;
+  a.m_tiles = (a.B + 128 * MT - 1) / (128 * MT);
+  a.n_tiles = a.H / C::U;
+  a.tiles = (int64_t)P * a.m_tiles * a.n_tiles;
+  cudaFuncSetAttribute(cell_tc_kernel<MT, BN, STAGES, ACC>,
+                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  const int64_t grid = a.tiles < sms ? a.tiles : sms;
+  cell_tc_kernel<MT, BN, STAGES, ACC><<<(int)grid, kTcThreads, C::SMEM, st>>>(A0, A1, Wm, a, P);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_cell_tc(const zo_ctx* ctx, int layer, int t, int B, int nprobe, int probe0,
+                           uint64_t seed, float eps, float* raw_out, cudaStream_t st) {
+  const zo_model_spec& s = ctx->spec;
+  const int H = s.hidden, E = s.embed;
+  const int P = 2 * nprobe;
+  const int K0 = layer == 0 ? E : H;
+  CellArgs a;
+  a.K0 = K0;
+  a.H = H;
+  a.Ktot = K0 + H;
+  a.nk = (t == 0 ? K0 : K0 + H) / 64;
+  a.B = B;
+  a.Bmax = s.max_batch;
+  a.group = 8;
+  a.seed = seed;
+  a.probe0 = probe0;
+  a.eps = eps;
+  a.offW = ctx->seg.off[ctx->seg.W[layer]];
+  a.small_p = ctx->small_p;
+  a.sstride = ctx->small.stride;
+  a.soffb = ctx->small.b[layer];
+  const int64_t PB = 2 * (int64_t)ctx->chunk * s.max_batch;
+  a.cst = ctx->cst + (int64_t)layer * PB * H;
+  a.hout = ctx->h + ((int64_t)layer * 2 + (t & 1)) * PB * H;
+  a.first = t == 0;
+  a.raw = raw_out;
+  a.err = ctx->err;
+  const CellMaps& m = *ctx->maps;
+  const CUtensorMap& A0 = layer == 0 ? m.x : m.h[layer - 1][t & 1];
+  const CUtensorMap& A1 = m.h[layer][(t + 1) & 1];
+  if (a.Ktot >= 4096)
+    return launch_cfg<2, kBN, 3, 1>(A0, A1, m.w[layer], a, P, ctx->sm_count, st);
+  return launch_cfg<1, kBN, 4, 2>(A0, A1, m.w[layer], a, P, ctx->sm_count, st);
+}
+
+}  // namespace zo

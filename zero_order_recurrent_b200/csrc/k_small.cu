@@ -1,0 +1,299 @@
+// Small kernels of the perturbed forward: perturbed copies of the small
+// segments, the embedding gather that builds the first layer's input, the
+// output projection with softmax cross-entropy, and the final per-probe loss
+// reduction.  "Central-difference random-vector gradient estimation evaluates
+// complete recurrent forwards at perturbed weights" (alex-wiki, "Method").
+#include "zo_common.cuh"
+#include "zo_internal.h"
+
+namespace zo {
+
+// ---------------------------------------------------------------------------
+// Perturbed small segments: for every probe-sign ps = 2*ci + s of the chunk,
+// small_p[ps] = theta_seg + (s ? -eps : +eps) * p_{probe0+ci} over the
+// embedding, every cell bias, W_out and b_out (fp32).
+// ---------------------------------------------------------------------------
+struct SmallArgs {
+  const float* theta;
+  float* out;
+  uint64_t seed;
+  int probe0;
+  int nprobe;
+  float eps;
+  int nparts;
+  int64_t src[kMaxSeg];   // theta offset of each part
+  int64_t dst[kMaxSeg];   // float offset inside one probe-sign's block
+  int64_t len[kMaxSeg];
+  int64_t stride;         // floats per probe-sign
+  int64_t blocks_per_probe;
+  int64_t part_blk0[kMaxSeg + 1];  // first 128-block index of each part (cumulative)
+};
+
+__global__ void perturb_small_kernel(const SmallArgs a) {
+  const int64_t total = a.blocks_per_probe * a.nprobe;
+  for (int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; t < total;
+       t += (int64_t)gridDim.x * blockDim.x) {
+    const int ci = (int)(t / a.blocks_per_probe);
+    int64_t rb = t - (int64_t)ci * a.blocks_per_probe;
+    int part = 0;
+    while (part + 1 < a.nparts && rb >= a.part_blk0[part + 1]) ++part;
+    const int64_t kb = rb - a.part_blk0[part];               // block within part
+    const int64_t j0 = a.src[part] + kb * 128;                // 128-aligned theta index
+    const int64_t n = min((int64_t)128, a.len[part] - kb * 128);
+    const uint4 w = sign_block(a.seed, (uint32_t)(a.probe0 + ci), (uint64_t)(j0 >> 7));
+    float* op = a.out + (int64_t)(2 * ci) * a.stride + a.dst[part] + kb * 128;
+    float* om = op + a.stride;
+    for (int e = 0; e < n; ++e) {
+      const float th = a.theta[j0 + e];
+      const float d = sign_bit(w, j0 + e) ? -a.eps : a.eps;
+      op[e] = th + d;
+      om[e] = th - d;
+    }
+  }
+}
+
+cudaError_t launch_perturb_small(const zo_ctx* ctx, const float* theta, uint64_t seed, int probe0,
+                                 int nprobe, float eps, cudaStream_t st) {
+  const Segments& s = ctx->seg;
+  const SmallLayout& sl = ctx->small;
+  const int L = ctx->spec.layers;
+  SmallArgs a;
+  a.theta = theta;
+  a.out = ctx->small_p;
+  a.seed = seed;
+  a.probe0 = probe0;
+  a.nprobe = nprobe;
+  a.eps = eps;
+  int np = 0;
+  auto add = [&](int seg, int64_t dst) {
+    a.src[np] = s.off[seg];
+    a.dst[np] = dst;
+    a.len[np] = s.numel[seg];
+    ++np;
+  };
+  add(s.E, sl.E);
+  for (int l = 0; l < L; ++l) add(s.b[l], sl.b[l]);
+  add(s.Wout, sl.Wout);
+  add(s.bout, sl.bout);
+  a.nparts = np;
+  int64_t cum = 0;
+  for (int i = 0; i < np; ++i) {
+    a.part_blk0[i] = cum;
+    cum += (a.len[i] + 127) / 128;
+  }
+  a.part_blk0[np] = cum;
+  a.blocks_per_probe = cum;
+  a.stride = sl.stride;
+  const int64_t total = cum * nprobe;
+  int64_t grid = (total + 127) / 128;
+  if (grid > 65535) grid = 65535;
+  perturb_small_kernel<<<(int)grid, 128, 0, st>>>(a);
+  count_launch();
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// x_t[ps][b][:] = bf16(E_perturbed[ps][token[b, t]][:])  (first layer input)
+// ---------------------------------------------------------------------------
+__global__ void gather_x_kernel(const float* __restrict__ small_p, int64_t stride, int64_t offE,
+                                const int32_t* __restrict__ tokens, int t, int B, int T, int Bmax,
+                                int E, int V, int P, __nv_bfloat16* __restrict__ x,
+                                unsigned* err) {
+  const int e8 = E / 8;
+  const int64_t total = (int64_t)P * B * e8;
+  for (int64_t k = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; k < total;
+       k += (int64_t)gridDim.x * blockDim.x) {
+    const int c = (int)(k % e8);
+    const int64_t pb = k / e8;
+    const int b = (int)(pb % B);
+    const int ps = (int)(pb / B);
+    int tok = tokens[(int64_t)b * T + t];
+    if (tok < 0 || tok >= V) {
+      latch(err, kErrBounds);
+      tok = 0;
+    }
+    const float4* src = reinterpret_cast<const float4*>(small_p + ps * stride + offE +
+                                                        (int64_t)tok * E + 8 * c);
+    const float4 u = src[0], v = src[1];
+    __nv_bfloat162 q0 = __floats2bfloat162_rn(u.x, u.y), q1 = __floats2bfloat162_rn(u.z, u.w);
+    __nv_bfloat162 q2 = __floats2bfloat162_rn(v.x, v.y), q3 = __floats2bfloat162_rn(v.z, v.w);
+    uint4 o;
+    o.x = *reinterpret_cast<uint32_t*>(&q0);
+    o.y = *reinterpret_cast<uint32_t*>(&q1);
+    o.z = *reinterpret_cast<uint32_t*>(&q2);
+    o.w = *reinterpret_cast<uint32_t*>(&q3);
+    reinterpret_cast<uint4*>(x + ((int64_t)ps * Bmax + b) * E)[c] = o;
+  }
+}
+
+cudaError_t launch_gather_x(const zo_ctx* ctx, const int32_t* tokens, int t, int B, int T,
+                            int nprobe, cudaStream_t st) {
+  const int E = ctx->spec.embed;
+  const int P = 2 * nprobe;
+  const int64_t total = (int64_t)P * B * (E / 8);
+  int64_t grid = (total + 255) / 256;
+  if (grid > (int64_t)ctx->sm_count * 16) grid = (int64_t)ctx->sm_count * 16;
+  gather_x_kernel<<<(int)grid, 256, 0, st>>>(ctx->small_p, ctx->small.stride, ctx->small.E,
+                                             tokens, t, B, T, ctx->spec.max_batch, E,
+                                             ctx->spec.vocab, P, ctx->x, ctx->err);
+  count_launch();
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Output projection + softmax cross-entropy for one timestep (bf16 path).
+// Per probe-sign ps: logits[b][v] = h[ps][b][:] . Wout_p[ps][v][:] + bout_p[ps][v];
+// rowloss[ps][b] += logsumexp(logits[b]) - logits[b][target] when scored.
+// CTA tile: 64 rows x 64 logits (V <= 64), K chunks of 32, 4x4 per thread.
+// ---------------------------------------------------------------------------
+constexpr int kLossRows = 64;
+constexpr int kLossCols = 64;
+constexpr int kLossK = 32;
+
+__global__ void __launch_bounds__(256) loss_bf16_kernel(
+    const __nv_bfloat16* __restrict__ h, const float* __restrict__ small_p, int64_t stride,
+    int64_t offW, int64_t offb, const int32_t* __restrict__ targets, int t, int B, int T,
+    int Bmax, int H, int V, float* __restrict__ rowloss, unsigned* err) {
+  __shared__ float As[kLossK][kLossRows + 4];
+  __shared__ float Bs[kLossK][kLossCols + 4];
+  __shared__ float logit[kLossRows][kLossCols + 1];
+  const int ps = blockIdx.y;
+  const int r0 = blockIdx.x * kLossRows;
+  const int tid = threadIdx.x;
+  const int tx = tid & 15, ty = tid >> 4;
+  const __nv_bfloat16* hp = h + (int64_t)ps * Bmax * H;
+  const float* W = small_p + ps * stride + offW;
+  float acc[4][4] = {};
+  for (int k0 = 0; k0 < H; k0 += kLossK) {
+    {  // A: 64 rows x 32 k, 8 bf16 per thread
+      const int row = tid >> 2, kk = (tid & 3) * 8;
+      float v[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+      if (r0 + row < B && k0 + kk + 8 <= H) {
+        const uint4 raw = *reinterpret_cast<const uint4*>(hp + (int64_t)(r0 + row) * H + k0 + kk);
+        const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(&raw);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = __bfloat162float(e[i]);
+      } else if (r0 + row < B) {
+        for (int i = 0; i < 8; ++i)
+          if (k0 + kk + i < H) v[i] = __bfloat162float(hp[(int64_t)(r0 + row) * H + k0 + kk + i]);
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) As[kk + i][row] = v[i];
+    }
+    {  // B: 64 logits x 32 k
+      const int col = tid >> 2, kk = (tid & 3) * 8;
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        Bs[kk + i][col] = (col < V && k0 + kk + i < H) ? W[(int64_t)col * H + k0 + kk + i] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int k = 0; k < kLossK; ++k) {
+      float a[4], b[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) a[i] = As[k][ty * 4 + i];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) b[j] = Bs[k][tx * 4 + j];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) logit[ty * 4 + i][tx * 4 + j] = acc[i][j];
+  __syncthreads();
+  if (tid < kLossRows) {
+    const int b = r0 + tid;
+    if (b < B) {
+      int tg = targets[(int64_t)b * T + t];
+      if (tg >= V || tg < -1) {
+        latch(err, kErrBounds);
+        tg = -1;
+      }
+      if (tg >= 0) {
+        const float* bo = small_p + ps * stride + offb;
+        float m = -INFINITY;
+        for (int v = 0; v < V; ++v) m = fmaxf(m, logit[tid][v] + bo[v]);
+        float s = 0.f;
+        for (int v = 0; v < V; ++v) s += expf(logit[tid][v] + bo[v] - m);
+        const float lse = m + logf(s);
+        rowloss[(int64_t)ps * Bmax + b] += lse - (logit[tid][tg] + bo[tg]);
+      }
+    }
+  }
+}
+
+cudaError_t launch_loss_bf16(const zo_ctx* ctx, const int32_t* targets, int t, int B, int T,
+                             int nprobe, cudaStream_t st) {
+  const int L = ctx->spec.layers, H = ctx->spec.hidden;
+  const int P = 2 * nprobe;
+  const int Bmax = ctx->spec.max_batch;
+  const __nv_bfloat16* htop =
+      ctx->h + ((int64_t)(L - 1) * 2 + (t & 1)) * (int64_t)(2 * ctx->chunk) * Bmax * H;
+  dim3 grid((B + kLossRows - 1) / kLossRows, P);
+  loss_bf16_kernel<<<grid, 256, 0, st>>>(htop, ctx->small_p, ctx->small.stride, ctx->small.Wout,
+                                         ctx->small.bout, targets, t, B, T, Bmax, H,
+                                         ctx->spec.vocab, ctx->rowloss, ctx->err);
+  count_launch();
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// L[ps] = sum_b rowloss[ps][b] / #scored; fixed-order tree reduction, one CTA
+// per probe-sign.  Also copies the row sums out when asked.
+// ---------------------------------------------------------------------------
+__global__ void reduce_losses_kernel(const float* __restrict__ rowloss, int Bmax,
+                                     const int32_t* __restrict__ targets, int B, int T, int V,
+                                     int probe0, float* lp, float* lm, float* row_out,
+                                     unsigned* err) {
+  __shared__ double ssum[256];
+  __shared__ int scount[256];
+  const int ps = blockIdx.x;
+  double s = 0.0;
+  int cnt = 0;
+  for (int b = threadIdx.x; b < B; b += blockDim.x) {
+    const float v = rowloss[(int64_t)ps * Bmax + b];
+    s += v;
+    if (row_out) row_out[((int64_t)(2 * probe0) + ps) * B + b] = v;
+  }
+  for (int64_t k = threadIdx.x; k < (int64_t)B * T; k += blockDim.x) {
+    const int tg = targets[k];
+    cnt += (tg >= 0 && tg < V);
+  }
+  ssum[threadIdx.x] = s;
+  scount[threadIdx.x] = cnt;
+  __syncthreads();
+  for (int w = blockDim.x / 2; w > 0; w >>= 1) {
+    if (threadIdx.x < w) {
+      ssum[threadIdx.x] += ssum[threadIdx.x + w];
+      scount[threadIdx.x] += scount[threadIdx.x + w];
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    const int n = scount[0];
+    const float L = n > 0 ? (float)(ssum[0] / n) : 0.f;
+    if (!isfinite(L)) latch(err, kErrNonfinite);
+    const int i = probe0 + ps / 2;
+    if (ps & 1)
+      lm[i] = L;
+    else
+      lp[i] = L;
+  }
+}
+
+cudaError_t launch_reduce_losses(const zo_ctx* ctx, const int32_t* targets, int B, int T,
+                                 int probe0, int nprobe, float* lp, float* lm, float* row_out,
+                                 cudaStream_t st) {
+  reduce_losses_kernel<<<2 * nprobe, 256, 0, st>>>(ctx->rowloss, ctx->spec.max_batch, targets, B,
+                                                   T, ctx->spec.vocab, probe0, lp, lm, row_out,
+                                                   ctx->err);
+  count_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace zo

@@ -1,0 +1,230 @@
+// Coefficients and the seed-replayed update (pith.science review, "What
+// carries the argument": Theta' = Theta - 1/(2 n_pert) sum_i (L+_i - L-_i) p_i;
+// alex-wiki "Method": theta' = theta - eta g_hat), plus the probe-sign test
+// hook and the bf16 shadow cast.
+#include "zo_common.cuh"
+#include "zo_internal.h"
+
+namespace zo {
+
+// ---------------------------------------------------------------------------
+// Sign words (test hook)
+// ---------------------------------------------------------------------------
+__global__ void sign_words_kernel(uint64_t seed, uint32_t probe, int64_t q0, int64_t n,
+                                  uint32_t* out) {
+  for (int64_t k = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; k < n;
+       k += (int64_t)gridDim.x * blockDim.x) {
+    const uint4 w = sign_block(seed, probe, (uint64_t)(q0 + k));
+    reinterpret_cast<uint4*>(out)[k] = w;
+  }
+}
+
+cudaError_t launch_sign_words(uint64_t seed, int probe, int64_t q0, int64_t n, uint32_t* out,
+                              cudaStream_t st) {
+  if (n <= 0) return cudaSuccess;
+  const int grid = (int)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
+  sign_words_kernel<<<grid, 256, 0, st>>>(seed, (uint32_t)probe, q0, n, out);
+  count_launch();
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// bf16 shadow of theta
+// ---------------------------------------------------------------------------
+__global__ void cast_shadow_kernel(const float4* __restrict__ th, uint2* __restrict__ sh,
+                                   int64_t n4) {
+  for (int64_t k = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; k < n4;
+       k += (int64_t)gridDim.x * blockDim.x) {
+    const float4 v = th[k];
+    __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y);
+    __nv_bfloat162 b = __floats2bfloat162_rn(v.z, v.w);
+    uint2 o;
+    o.x = *reinterpret_cast<uint32_t*>(&a);
+    o.y = *reinterpret_cast<uint32_t*>(&b);
+    sh[k] = o;
+  }
+}
+
+cudaError_t launch_cast_shadow(const float* theta, __nv_bfloat16* shadow, int64_t d_pad,
+                               cudaStream_t st) {
+  const int64_t n4 = d_pad / 4;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  int64_t grid = (n4 + 255) / 256;
+  if (grid > (int64_t)sms * 8) grid = (int64_t)sms * 8;
+  if (grid < 1) grid = 1;
+  cast_shadow_kernel<<<(int)grid, 256, 0, st>>>(reinterpret_cast<const float4*>(theta),
+                                                 reinterpret_cast<uint2*>(shadow), n4);
+  count_launch();
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Coefficients c_i = eta (L+_i - L-_i) / (2 eps n_pert)
+// ---------------------------------------------------------------------------
+__global__ void coeffs_kernel(const float* lp, const float* lm, int n, float eps, float eta,
+                              float* out, unsigned* err) {
+  const float scale = eta / (2.f * eps * (float)n);
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+    const float a = lp[i], b = lm[i];
+    float c = (a - b) * scale;
+    if (!isfinite(a) || !isfinite(b) || !isfinite(c)) {
+      latch(err, kErrNonfinite);
+      c = __int_as_float(0x7fc00000);
+    }
+    out[i] = c;
+  }
+}
+
+cudaError_t launch_coeffs(const float* lp, const float* lm, int n, float eps, float eta,
+                          float* out, unsigned* err, cudaStream_t st) {
+  const int grid = (n + 255) / 256;
+  coeffs_kernel<<<grid, 256, 0, st>>>(lp, lm, n, eps, eta, out, err);
+  count_launch();
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Update.  One warp handles a span of 32 blocks (4096 parameters).  In the
+// sign phase lane L computes the Philox block for block L of the span, once
+// per probe, and parks the words in shared memory; in the apply phase the
+// warp walks the span block by block, lane L owning the float4 at 4L..4L+3,
+// so every global access is a coalesced 512-byte row.  Probes are summed in
+// fp32 groups of 8 and the groups in fp64, then theta is rounded once.
+// More than kUpdProbes probes are applied in successive passes over the span.
+// ---------------------------------------------------------------------------
+constexpr int kUpdWarps = 4;
+constexpr int kUpdProbes = 32;
+constexpr int kUpdBatch = 4;   // blocks whose theta is loaded ahead
+
+struct UpdateArgs {
+  float* theta;
+  __nv_bfloat16* shadow;   // may be null
+  const float* coeffs;
+  uint64_t seed;
+  int n;
+  int64_t nblk;            // d_pad / 128
+  int nseg;
+  int64_t seg_off[kMaxSeg];
+  int64_t seg_end[kMaxSeg];
+  unsigned* err;
+};
+
+__device__ __forceinline__ int64_t real_end_of(const UpdateArgs& a, int64_t j) {
+  int64_t end = a.seg_end[0];
+#pragma unroll 1
+  for (int s = 0; s < a.nseg; ++s)
+    if (j >= a.seg_off[s]) end = a.seg_end[s];
+  return end;
+}
+
+__global__ void __launch_bounds__(kUpdWarps * 32) update_kernel(const UpdateArgs a) {
+  extern __shared__ uint4 words_sm[];  // [kUpdWarps][kUpdProbes][32]
+  __shared__ int bad;
+  if (threadIdx.x == 0) bad = 0;
+  __syncthreads();
+  for (int i = threadIdx.x; i < a.n; i += blockDim.x)
+    if (!isfinite(a.coeffs[i])) bad = 1;
+  __syncthreads();
+  if (bad) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) latch(a.err, kErrNonfinite);
+    return;
+  }
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  uint4* words = words_sm + warp * kUpdProbes * 32;
+  const int64_t nspan = (a.nblk + 31) / 32;
+  const int64_t gw = blockIdx.x * (int64_t)kUpdWarps + warp;
+  const int64_t nw = (int64_t)gridDim.x * kUpdWarps;
+  const int widx = lane >> 3;
+  const int sh = 2 * (lane & 7);
+
+  for (int64_t span = gw; span < nspan; span += nw) {
+    const int64_t q0 = span * 32;
+    const int nq = (int)min((int64_t)32, a.nblk - q0);
+    for (int p0 = 0; p0 < a.n; p0 += kUpdProbes) {
+      const int np = min(kUpdProbes, a.n - p0);
+      const bool last_pass = p0 + kUpdProbes >= a.n;
+      if (lane < nq)
+        for (int i = 0; i < np; ++i)
+          words[i * 32 + lane] = sign_block(a.seed, (uint32_t)(p0 + i), (uint64_t)(q0 + lane));
+      __syncwarp();
+      for (int it0 = 0; it0 < nq; it0 += kUpdBatch) {
+        float4 th[kUpdBatch];
+#pragma unroll
+        for (int u = 0; u < kUpdBatch; ++u)
+          if (it0 + u < nq)
+            th[u] = reinterpret_cast<const float4*>(a.theta)[(q0 + it0 + u) * 32 + lane];
+#pragma unroll
+        for (int u = 0; u < kUpdBatch; ++u) {
+          const int it = it0 + u;
+          if (it >= nq) break;
+          double acc0 = th[u].x, acc1 = th[u].y, acc2 = th[u].z, acc3 = th[u].w;
+          const uint32_t* wcol = reinterpret_cast<const uint32_t*>(words + it) + widx;
+          for (int g = 0; g < np; g += 8) {
+            float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+            const int ge = min(g + 8, np);
+            for (int i = g; i < ge; ++i) {
+              const float nc = -__ldg(a.coeffs + p0 + i);
+              const uint32_t w = wcol[i * 32 * 4] >> sh;
+              s0 += flip_sign(nc, w << 31);
+              s1 += flip_sign(nc, w << 15);
+              s2 += flip_sign(nc, w << 30);
+              s3 += flip_sign(nc, w << 14);
+            }
+            acc0 += s0;
+            acc1 += s1;
+            acc2 += s2;
+            acc3 += s3;
+          }
+          const int64_t j = (q0 + it) * 128 + 4 * lane;
+          const int64_t lim = real_end_of(a, (q0 + it) * 128);
+          float4 o;
+          o.x = j + 0 < lim ? (float)acc0 : th[u].x;
+          o.y = j + 1 < lim ? (float)acc1 : th[u].y;
+          o.z = j + 2 < lim ? (float)acc2 : th[u].z;
+          o.w = j + 3 < lim ? (float)acc3 : th[u].w;
+          reinterpret_cast<float4*>(a.theta)[(q0 + it) * 32 + lane] = o;
+          if (last_pass && a.shadow) {
+            __nv_bfloat162 lo = __floats2bfloat162_rn(o.x, o.y);
+            __nv_bfloat162 hi = __floats2bfloat162_rn(o.z, o.w);
+            uint2 pk;
+            pk.x = *reinterpret_cast<uint32_t*>(&lo);
+            pk.y = *reinterpret_cast<uint32_t*>(&hi);
+            reinterpret_cast<uint2*>(a.shadow)[(q0 + it) * 32 + lane] = pk;
+          }
+        }
+      }
+      __syncwarp();
+    }
+  }
+}
+
+cudaError_t launch_update(const zo_ctx* ctx, float* theta, uint64_t seed, int n,
+                          const float* coeffs, __nv_bfloat16* shadow, cudaStream_t st) {
+  UpdateArgs a;
+  a.theta = theta;
+  a.shadow = shadow;
+  a.coeffs = coeffs;
+  a.seed = seed;
+  a.n = n;
+  a.nblk = ctx->seg.d_pad / 128;
+  a.nseg = ctx->seg.n;
+  for (int s = 0; s < ctx->seg.n; ++s) {
+    a.seg_off[s] = ctx->seg.off[s];
+    a.seg_end[s] = ctx->seg.off[s] + ctx->seg.numel[s];
+  }
+  a.err = ctx->err;
+  const size_t smem = sizeof(uint4) * kUpdWarps * kUpdProbes * 32;
+  cudaFuncSetAttribute(update_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  const int64_t nspan = (a.nblk + 31) / 32;
+  int64_t grid = (nspan + kUpdWarps - 1) / kUpdWarps;
+  const int64_t cap = (int64_t)ctx->sm_count * 3;
+  if (grid > cap) grid = cap;
+  update_kernel<<<(int)grid, kUpdWarps * 32, smem, st>>>(a);
+  count_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace zo

@@ -1,0 +1,116 @@
+// Host-side internals shared by the library's translation units: the
+// context, its workspace and the kernel launchers.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include <atomic>
+#include <vector>
+
+#include "../../include/zo.h"
+
+namespace zo {
+
+constexpr int kMaxLayersHost = 8;
+constexpr int kMaxSegHost = 2 + 2 * kMaxLayersHost;
+
+// Segment table in the flat parameter vector.
+struct Segments {
+  int n = 0;
+  int64_t off[kMaxSegHost];
+  int64_t numel[kMaxSegHost];
+  int64_t d_pad = 0, d_real = 0;
+  // indices into off/numel
+  int E = 0, W[kMaxLayersHost], b[kMaxLayersHost], Wout = 0, bout = 0;
+};
+
+// Per-probe-sign perturbed copies of the small segments (bf16 path):
+// embedding, cell biases, output weights and bias, fp32.
+struct SmallLayout {
+  int64_t E = 0, b[kMaxLayersHost], Wout = 0, bout = 0, stride = 0;  // float offsets
+};
+
+struct CellMaps {
+  alignas(64) CUtensorMap x;                    // x_t            [P][B][E]  bf16
+  alignas(64) CUtensorMap h[kMaxLayersHost][2];  // h_l (parity)   [P][B][H]  bf16
+  alignas(64) CUtensorMap w[kMaxLayersHost];     // W_l shadow     [4H][in+H] bf16
+};
+
+}  // namespace zo
+
+struct ZoProfRec {
+  cudaEvent_t a = nullptr, b = nullptr;
+  int kind = 0;
+  double flops = 0, bytes = 0;
+};
+
+struct zo_ctx {
+  zo_model_spec spec;
+  int device = 0;
+  int sm_count = 0;
+  zo::Segments seg;
+  int chunk = 0;            // probes per pass
+  int64_t ws_bytes = 0;
+  unsigned* err = nullptr;  // device error word
+  // bf16 path
+  __nv_bfloat16* shadow = nullptr;
+  const float* shadow_theta = nullptr;
+  bool shadow_fresh = false;
+  zo::SmallLayout small;
+  float* small_p = nullptr;      // [2*chunk][small.stride]
+  __nv_bfloat16* x = nullptr;    // [2*chunk][B][E]
+  __nv_bfloat16* h = nullptr;    // [L][2][2*chunk][B][H]
+  float* cst = nullptr;          // [L][2*chunk][B][H]
+  zo::CellMaps* maps = nullptr;  // host copy of the tensor maps
+  // both paths
+  float* rowloss = nullptr;      // [2*chunk][B]
+  // zo_step_host staging (device)
+  int32_t* tok = nullptr;
+  int32_t* tgt = nullptr;
+  float* lp = nullptr;
+  float* lm = nullptr;
+  float* coef = nullptr;
+  int n_stage = 0;               // capacity of lp/lm/coef
+  int fp32_bb = 1;               // rows per CTA of the fp32 forward
+  size_t fp32_smem = 0;
+  // per-launch timing (zo_profile)
+  bool prof_on = false;
+  std::vector<ZoProfRec> prof;
+  size_t prof_used = 0;
+};
+
+namespace zo {
+
+extern std::atomic<int64_t> g_launches;
+inline void count_launch(int n = 1) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+// ---- launchers (each returns cudaGetLastError() after enqueueing) ----
+cudaError_t launch_sign_words(uint64_t seed, int probe, int64_t q0, int64_t n, uint32_t* out,
+                              cudaStream_t st);
+cudaError_t launch_cast_shadow(const float* theta, __nv_bfloat16* shadow, int64_t d_pad,
+                               cudaStream_t st);
+cudaError_t launch_coeffs(const float* lp, const float* lm, int n, float eps, float eta,
+                          float* out, unsigned* err, cudaStream_t st);
+cudaError_t launch_update(const zo_ctx* ctx, float* theta, uint64_t seed, int n,
+                          const float* coeffs, __nv_bfloat16* shadow, cudaStream_t st);
+cudaError_t launch_fp32_forward(const zo_ctx* ctx, const float* theta, uint64_t seed, int probe0,
+                                int nprobe, float eps, const int32_t* tokens,
+                                const int32_t* targets, int B, int T, cudaStream_t st);
+cudaError_t launch_reduce_losses(const zo_ctx* ctx, const int32_t* targets, int B, int T,
+                                 int probe0, int nprobe, float* lp, float* lm, float* row_out,
+                                 cudaStream_t st);
+// bf16 path
+cudaError_t launch_perturb_small(const zo_ctx* ctx, const float* theta, uint64_t seed, int probe0,
+                                 int nprobe, float eps, cudaStream_t st);
+cudaError_t launch_gather_x(const zo_ctx* ctx, const int32_t* tokens, int t, int B, int T,
+                            int nprobe, cudaStream_t st);
+cudaError_t launch_loss_bf16(const zo_ctx* ctx, const int32_t* targets, int t, int B, int T,
+                             int nprobe, cudaStream_t st);
+cudaError_t launch_cell_tc(const zo_ctx* ctx, int layer, int t, int B, int nprobe, int probe0,
+                           uint64_t seed, float eps, float* raw_out, cudaStream_t st);
+bool make_cell_maps(zo_ctx* ctx);
+
+}  // namespace zo
