@@ -12,10 +12,11 @@
 // CTA tile: MT sub-tiles of 128 batch rows x BN gate rows (BN/4 hidden units,
 // the four gate blocks side by side so the epilogue sees i, f, g, o of a unit
 // together) x 64-deep K stages.  Warp roles (320 threads):
-//   warp 0      TMA producer (A activations, W_l tile as 4 gate boxes)
-//   warp 1      TMEM allocator and MMA issuer
-//   warps 2..5  perturbation: W tile += +-eps p in shared memory
-//   warps 6..9  epilogue: TMEM -> gates -> c, h (TMEM lane quadrant = warp % 4)
+//   warp 0       TMA producer (A activations, W_l tile as 4 gate boxes)
+//   warp 1       TMEM allocator and MMA issuer
+//   warps 2..9   perturbation: W tile += +-eps p in shared memory, one row
+//                per thread, two warps per SM sub-partition to hide latency
+//   warps 10..13 epilogue: TMEM -> gates -> c, h (TMEM lane quadrant = warp % 4)
 // Every mbarrier wait is bounded: past ~2 s the CTA raises an abort flag, the
 // error word gets ZO_ERR_TIMEOUT, all roles leave their loops, and tensor
 // memory is freed before exit.  No multicast form of any copy is used.
@@ -26,7 +27,9 @@
 
 namespace zo {
 
-constexpr int kTcThreads = 320;
+constexpr int kTcThreads = 448;
+constexpr int kGenThreads = 256;
+constexpr int kGenWarps = kGenThreads / 32;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
 struct CellArgs {
@@ -181,6 +184,13 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
       : "r"(taddr));
 }
 
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                 "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+}
+
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -262,7 +272,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(full_bar(s), 1);
-      mbar_init(ready_bar(s), 4);
+      mbar_init(ready_bar(s), kGenWarps);
       mbar_init(empty_bar(s), 1);
     }
     for (int b = 0; b < ACC; ++b) {
@@ -379,10 +389,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       while (!mbar_try(drain_bar, 0) && globaltimer() - t0 < 100000000ull) {
       }
     }
-  } else if (warp < 6) {
+  } else if (warp < 2 + kGenWarps) {
     // ------------------------------------------------------------ perturbation
-    const int gt = threadIdx.x - 64;  // 0..127
-    constexpr int RPT = BN / 128 > 0 ? BN / 128 : 1;
+    const int gt = threadIdx.x - 64;  // 0..kGenThreads-1
+    constexpr int RPT = (BN + kGenThreads - 1) / kGenThreads;
     const float epsf = a.eps;
     const __nv_bfloat16 eb = __float2bfloat16_rn(epsf);
     const uint32_t eps_bits = (uint32_t)(*reinterpret_cast<const uint16_t*>(&eb));
@@ -408,7 +418,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         uint8_t* tileB = smem + s * C::STAGE + C::A_BYTES;
 #pragma unroll
         for (int rr = 0; rr < RPT; ++rr) {
-          const int r = gt + rr * 128;
+          const int r = gt + rr * kGenThreads;
           if (r < BN) {
             const int g = r / C::U, u = r % C::U;
             const int64_t R = (int64_t)g * a.H + (int64_t)tc.n * C::U + u;
@@ -460,22 +470,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const int b = tc.m * 128 * MT + mt * 128 + rloc;
         const int64_t rowoff = ((int64_t)tc.ps * a.Bmax + b) * a.H;
 #pragma unroll 1
-        for (int u0 = 0; u0 < C::U; u0 += 16) {
-          uint32_t acc[4][16];
+        for (int u0 = 0; u0 < C::U; u0 += 8) {
+          uint32_t acc[4][8];
 #pragma unroll
           for (int g = 0; g < 4; ++g)
-            tmem_ld16(tmem_base + ((uint32_t)(quad * 32) << 16) + ab * C::COLS + mt * BN +
-                          g * C::U + u0,
-                      acc[g]);
+            tmem_ld8(tmem_base + ((uint32_t)(quad * 32) << 16) + ab * C::COLS + mt * BN +
+                         g * C::U + u0,
+                     acc[g]);
           tmem_wait_ld();
           if (b < a.B) {
             const int unit0 = tc.n * C::U + u0;
-            float pre[4][16];
+            float pre[4][8];
 #pragma unroll
             for (int g = 0; g < 4; ++g) {
               const float4* bp = reinterpret_cast<const float4*>(bias + g * a.H + unit0);
 #pragma unroll
-              for (int q4 = 0; q4 < 4; ++q4) {
+              for (int q4 = 0; q4 < 2; ++q4) {
                 const float4 bv = __ldg(bp + q4);
                 pre[g][4 * q4 + 0] = __uint_as_float(acc[g][4 * q4 + 0]) + bv.x;
                 pre[g][4 * q4 + 1] = __uint_as_float(acc[g][4 * q4 + 1]) + bv.y;
@@ -488,19 +498,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
               for (int g = 0; g < 4; ++g)
 #pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4)
+                for (int q4 = 0; q4 < 2; ++q4)
                   reinterpret_cast<float4*>(rp + g * a.H + unit0)[q4] =
                       make_float4(pre[g][4 * q4], pre[g][4 * q4 + 1], pre[g][4 * q4 + 2],
                                   pre[g][4 * q4 + 3]);
             } else {
-              float cprev[16];
+              float cprev[8];
               float4* cp = reinterpret_cast<float4*>(a.cst + rowoff + unit0);
               if (a.first) {
 #pragma unroll
-                for (int i = 0; i < 16; ++i) cprev[i] = 0.f;
+                for (int i = 0; i < 8; ++i) cprev[i] = 0.f;
               } else {
 #pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
+                for (int q4 = 0; q4 < 2; ++q4) {
                   const float4 v = cp[q4];
                   cprev[4 * q4] = v.x;
                   cprev[4 * q4 + 1] = v.y;
@@ -508,30 +518,27 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                   cprev[4 * q4 + 3] = v.w;
                 }
               }
-              float cn[16];
-              uint32_t hp[8];
+              float cn[8];
+              uint32_t hp[4];
 #pragma unroll
-              for (int i = 0; i < 16; ++i) {
-                const float ig = sigmoid_fast(pre[0][i]);
-                const float fg = sigmoid_fast(pre[1][i]);
-                const float gg = tanh_fast(pre[2][i]);
-                const float og = sigmoid_fast(pre[3][i]);
-                cn[i] = fmaf(fg, cprev[i], ig * gg);
-                const float hv = og * tanh_fast(cn[i]);
-                if (i & 1) {
-                  __nv_bfloat162 pr = __floats2bfloat162_rn(
-                      __uint_as_float(hp[i >> 1]), hv);
-                  hp[i >> 1] = *reinterpret_cast<uint32_t*>(&pr);
-                } else {
-                  hp[i >> 1] = __float_as_uint(hv);
+              for (int i = 0; i < 8; i += 2) {
+                float hv[2];
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                  const float ig = sigmoid_fast(pre[0][i + e]);
+                  const float fg = sigmoid_fast(pre[1][i + e]);
+                  const float gg = tanh_fast(pre[2][i + e]);
+                  const float og = sigmoid_fast(pre[3][i + e]);
+                  cn[i + e] = fmaf(fg, cprev[i + e], ig * gg);
+                  hv[e] = og * tanh_fast(cn[i + e]);
                 }
+                __nv_bfloat162 pr = __floats2bfloat162_rn(hv[0], hv[1]);
+                hp[i >> 1] = *reinterpret_cast<uint32_t*>(&pr);
               }
 #pragma unroll
-              for (int q4 = 0; q4 < 4; ++q4)
+              for (int q4 = 0; q4 < 2; ++q4)
                 cp[q4] = make_float4(cn[4 * q4], cn[4 * q4 + 1], cn[4 * q4 + 2], cn[4 * q4 + 3]);
-              uint4* hq = reinterpret_cast<uint4*>(a.hout + rowoff + unit0);
-              hq[0] = make_uint4(hp[0], hp[1], hp[2], hp[3]);
-              hq[1] = make_uint4(hp[4], hp[5], hp[6], hp[7]);
+              *reinterpret_cast<uint4*>(a.hout + rowoff + unit0) = make_uint4(hp[0], hp[1], hp[2], hp[3]);
             }
           }
         }

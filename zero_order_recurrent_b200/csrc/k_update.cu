@@ -86,17 +86,18 @@ cudaError_t launch_coeffs(const float* lp, const float* lm, int n, float eps, fl
 }
 
 // ---------------------------------------------------------------------------
-// Update.  One warp handles a span of 32 blocks (4096 parameters).  In the
-// sign phase lane L computes the Philox block for block L of the span, once
-// per probe, and parks the words in shared memory; in the apply phase the
+// Update.  One warp handles a span of S consecutive 128-element blocks.  In
+// the sign phase the 32 lanes compute the Philox words of all (probe, block)
+// pairs of the span and park them in shared memory; in the apply phase the
 // warp walks the span block by block, lane L owning the float4 at 4L..4L+3,
 // so every global access is a coalesced 512-byte row.  Probes are summed in
-// fp32 groups of 8 and the groups in fp64, then theta is rounded once.
-// More than kUpdProbes probes are applied in successive passes over the span.
+// fp32 groups of 8 and the groups in fp64, then theta is rounded once.  S is
+// chosen on the host so that all probes fit one pass (S * probes <= 512
+// words per warp) and the spans still fill the GPU; with more probes than
+// that, successive passes re-read theta.
 // ---------------------------------------------------------------------------
 constexpr int kUpdWarps = 4;
-constexpr int kUpdProbes = 32;
-constexpr int kUpdBatch = 4;   // blocks whose theta is loaded ahead
+constexpr int kUpdSlots = 512;   // uint4 sign-word slots per warp (8 KB)
 
 struct UpdateArgs {
   float* theta;
@@ -105,27 +106,26 @@ struct UpdateArgs {
   uint64_t seed;
   int n;
   int64_t nblk;            // d_pad / 128
+  int S;                   // blocks per span
+  int pmax;                // probes per pass (pmax * S <= kUpdSlots)
   int nseg;
   int64_t seg_off[kMaxSeg];
   int64_t seg_end[kMaxSeg];
   unsigned* err;
 };
 
-__device__ __forceinline__ int64_t real_end_of(const UpdateArgs& a, int64_t j) {
-  int64_t end = a.seg_end[0];
-#pragma unroll 1
-  for (int s = 0; s < a.nseg; ++s)
-    if (j >= a.seg_off[s]) end = a.seg_end[s];
-  return end;
-}
-
 __global__ void __launch_bounds__(kUpdWarps * 32) update_kernel(const UpdateArgs a) {
-  extern __shared__ uint4 words_sm[];  // [kUpdWarps][kUpdProbes][32]
+  extern __shared__ uint4 dyn[];
+  float* negc = reinterpret_cast<float*>(dyn);             // [n], padded to 4
+  uint4* words_all = dyn + (a.n + 3) / 4;                   // [warps][kUpdSlots]
   __shared__ int bad;
   if (threadIdx.x == 0) bad = 0;
   __syncthreads();
-  for (int i = threadIdx.x; i < a.n; i += blockDim.x)
-    if (!isfinite(a.coeffs[i])) bad = 1;
+  for (int i = threadIdx.x; i < a.n; i += blockDim.x) {
+    const float c = a.coeffs[i];
+    if (!isfinite(c)) bad = 1;
+    negc[i] = -c;
+  }
   __syncthreads();
   if (bad) {
     if (blockIdx.x == 0 && threadIdx.x == 0) latch(a.err, kErrNonfinite);
@@ -133,67 +133,73 @@ __global__ void __launch_bounds__(kUpdWarps * 32) update_kernel(const UpdateArgs
   }
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
-  uint4* words = words_sm + warp * kUpdProbes * 32;
-  const int64_t nspan = (a.nblk + 31) / 32;
+  uint4* words = words_all + warp * kUpdSlots;
+  const uint32_t* words32 = reinterpret_cast<const uint32_t*>(words);
+  const int S = a.S;
+  const int64_t nspan = (a.nblk + S - 1) / S;
   const int64_t gw = blockIdx.x * (int64_t)kUpdWarps + warp;
   const int64_t nw = (int64_t)gridDim.x * kUpdWarps;
   const int widx = lane >> 3;
   const int sh = 2 * (lane & 7);
+  const float4* th4 = reinterpret_cast<const float4*>(a.theta);
 
   for (int64_t span = gw; span < nspan; span += nw) {
-    const int64_t q0 = span * 32;
-    const int nq = (int)min((int64_t)32, a.nblk - q0);
-    for (int p0 = 0; p0 < a.n; p0 += kUpdProbes) {
-      const int np = min(kUpdProbes, a.n - p0);
-      const bool last_pass = p0 + kUpdProbes >= a.n;
-      if (lane < nq)
-        for (int i = 0; i < np; ++i)
-          words[i * 32 + lane] = sign_block(a.seed, (uint32_t)(p0 + i), (uint64_t)(q0 + lane));
+    const int64_t q0 = span * S;
+    const int nq = (int)min((int64_t)S, a.nblk - q0);
+    // segment of the span's first block; segments start on block boundaries
+    int seg = 0;
+    while (seg + 1 < a.nseg && q0 * 128 >= a.seg_off[seg + 1]) ++seg;
+    for (int p0 = 0; p0 < a.n; p0 += a.pmax) {
+      const int np = min(a.pmax, a.n - p0);
+      const bool last_pass = p0 + a.pmax >= a.n;
+      const int pairs = np * S;
+#pragma unroll 4
+      for (int t = lane; t < pairs; t += 32) {
+        const int i = t / S, b = t - i * S;
+        if (b < nq) words[t] = sign_block(a.seed, (uint32_t)(p0 + i), (uint64_t)(q0 + b));
+      }
       __syncwarp();
-      for (int it0 = 0; it0 < nq; it0 += kUpdBatch) {
-        float4 th[kUpdBatch];
-#pragma unroll
-        for (int u = 0; u < kUpdBatch; ++u)
-          if (it0 + u < nq)
-            th[u] = reinterpret_cast<const float4*>(a.theta)[(q0 + it0 + u) * 32 + lane];
-#pragma unroll
-        for (int u = 0; u < kUpdBatch; ++u) {
-          const int it = it0 + u;
-          if (it >= nq) break;
-          double acc0 = th[u].x, acc1 = th[u].y, acc2 = th[u].z, acc3 = th[u].w;
-          const uint32_t* wcol = reinterpret_cast<const uint32_t*>(words + it) + widx;
-          for (int g = 0; g < np; g += 8) {
-            float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-            const int ge = min(g + 8, np);
-            for (int i = g; i < ge; ++i) {
-              const float nc = -__ldg(a.coeffs + p0 + i);
-              const uint32_t w = wcol[i * 32 * 4] >> sh;
-              s0 += flip_sign(nc, w << 31);
-              s1 += flip_sign(nc, w << 15);
-              s2 += flip_sign(nc, w << 30);
-              s3 += flip_sign(nc, w << 14);
-            }
-            acc0 += s0;
-            acc1 += s1;
-            acc2 += s2;
-            acc3 += s3;
+      int sg = seg;
+      float4 nxt = th4[q0 * 32 + lane];
+      for (int it = 0; it < nq; ++it) {
+        const int64_t q = q0 + it;
+        const float4 th = nxt;
+        if (it + 1 < nq) nxt = th4[(q + 1) * 32 + lane];
+        double acc0 = th.x, acc1 = th.y, acc2 = th.z, acc3 = th.w;
+        const uint32_t* wcol = words32 + it * 4 + widx;
+        for (int g = 0; g < np; g += 8) {
+          float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+          const int ge = min(g + 8, np);
+#pragma unroll 8
+          for (int i = g; i < ge; ++i) {
+            const float nc = negc[p0 + i];
+            const uint32_t w = wcol[i * S * 4] >> sh;
+            s0 += flip_sign(nc, w << 31);
+            s1 += flip_sign(nc, w << 15);
+            s2 += flip_sign(nc, w << 30);
+            s3 += flip_sign(nc, w << 14);
           }
-          const int64_t j = (q0 + it) * 128 + 4 * lane;
-          const int64_t lim = real_end_of(a, (q0 + it) * 128);
-          float4 o;
-          o.x = j + 0 < lim ? (float)acc0 : th[u].x;
-          o.y = j + 1 < lim ? (float)acc1 : th[u].y;
-          o.z = j + 2 < lim ? (float)acc2 : th[u].z;
-          o.w = j + 3 < lim ? (float)acc3 : th[u].w;
-          reinterpret_cast<float4*>(a.theta)[(q0 + it) * 32 + lane] = o;
-          if (last_pass && a.shadow) {
-            __nv_bfloat162 lo = __floats2bfloat162_rn(o.x, o.y);
-            __nv_bfloat162 hi = __floats2bfloat162_rn(o.z, o.w);
-            uint2 pk;
-            pk.x = *reinterpret_cast<uint32_t*>(&lo);
-            pk.y = *reinterpret_cast<uint32_t*>(&hi);
-            reinterpret_cast<uint2*>(a.shadow)[(q0 + it) * 32 + lane] = pk;
-          }
+          acc0 += s0;
+          acc1 += s1;
+          acc2 += s2;
+          acc3 += s3;
+        }
+        while (sg + 1 < a.nseg && q * 128 >= a.seg_off[sg + 1]) ++sg;
+        const int64_t j = q * 128 + 4 * lane;
+        const int64_t lim = a.seg_end[sg];
+        float4 o;
+        o.x = j + 0 < lim ? (float)acc0 : th.x;
+        o.y = j + 1 < lim ? (float)acc1 : th.y;
+        o.z = j + 2 < lim ? (float)acc2 : th.z;
+        o.w = j + 3 < lim ? (float)acc3 : th.w;
+        reinterpret_cast<float4*>(a.theta)[q * 32 + lane] = o;
+        if (last_pass && a.shadow) {
+          __nv_bfloat162 lo = __floats2bfloat162_rn(o.x, o.y);
+          __nv_bfloat162 hi = __floats2bfloat162_rn(o.z, o.w);
+          uint2 pk;
+          pk.x = *reinterpret_cast<uint32_t*>(&lo);
+          pk.y = *reinterpret_cast<uint32_t*>(&hi);
+          reinterpret_cast<uint2*>(a.shadow)[q * 32 + lane] = pk;
         }
       }
       __syncwarp();
@@ -216,11 +222,22 @@ cudaError_t launch_update(const zo_ctx* ctx, float* theta, uint64_t seed, int n,
     a.seg_end[s] = ctx->seg.off[s] + ctx->seg.numel[s];
   }
   a.err = ctx->err;
-  const size_t smem = sizeof(uint4) * kUpdWarps * kUpdProbes * 32;
+  // blocks per span: all probes in one pass if possible, and enough spans
+  // to give every SM 16 warps of work
+  int S = 32;
+  while (S > 1 && S * n > kUpdSlots) S /= 2;
+  const int64_t want = (int64_t)ctx->sm_count * 16;
+  while (S > 1 && (a.nblk + S - 1) / S < want) S /= 2;
+  a.S = S;
+  a.pmax = kUpdSlots / S < n ? kUpdSlots / S : n;
+  const size_t smem = sizeof(uint4) * ((n + 3) / 4 + (size_t)kUpdWarps * kUpdSlots);
   cudaFuncSetAttribute(update_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  const int64_t nspan = (a.nblk + 31) / 32;
+  const int64_t nspan = (a.nblk + S - 1) / S;
   int64_t grid = (nspan + kUpdWarps - 1) / kUpdWarps;
-  const int64_t cap = (int64_t)ctx->sm_count * 3;
+  int per_sm = (int)((200 * 1024) / smem);
+  if (per_sm < 1) per_sm = 1;
+  if (per_sm > 8) per_sm = 8;
+  const int64_t cap = (int64_t)ctx->sm_count * per_sm;
   if (grid > cap) grid = cap;
   update_kernel<<<(int)grid, kUpdWarps * 32, smem, st>>>(a);
   count_launch();

@@ -15,7 +15,7 @@
 
 namespace zo {
 std::atomic<int64_t> g_launches{0};
-size_t fp32_smem_bytes(const zo_model_spec& s, int bb);
+size_t fp32_smem_bytes(const zo_model_spec& s, int bb, int64_t d_pad);
 }  // namespace zo
 
 using namespace zo;
@@ -175,14 +175,16 @@ int zo_create(const zo_model_spec* spec, zo_ctx** out) {
 
   if (s.dtype == ZO_DTYPE_FP32) {
     // rows per CTA: the smallest power of two >= min(B, 8) whose state fits
+    // (the probe's sign words for all d_pad parameters live in shared memory)
+    const int64_t dp = c->seg.d_pad;
     int bb = 8;
-    while (bb > 1 && (bb / 2 >= B || fp32_smem_bytes(s, bb) > 200 * 1024)) bb /= 2;
-    if (fp32_smem_bytes(s, bb) > 200 * 1024) {
+    while (bb > 1 && (bb / 2 >= B || fp32_smem_bytes(s, bb, dp) > 200 * 1024)) bb /= 2;
+    if (fp32_smem_bytes(s, bb, dp) > 200 * 1024) {
       free_ctx(c);
       return ZO_ERR_UNSUPPORTED;
     }
     c->fp32_bb = bb;
-    c->fp32_smem = fp32_smem_bytes(s, bb);
+    c->fp32_smem = fp32_smem_bytes(s, bb, dp);
     c->chunk = s.chunk > 0 ? s.chunk : 4096;
     alloc((void**)&c->rowloss, sizeof(float) * 2 * (size_t)c->chunk * B);
   } else {
