@@ -330,3 +330,37 @@ def test_bf16_charlm_full_size_two_probes():
     assert np.allclose(lp[probes], olp, rtol=1e-2) and np.allclose(lm[probes], olm, rtol=1e-2)
     assert sign_agreement(lp[probes], lm[probes], olp, olm) >= 0.95
     assert estimate_cosine(spec_of(cfg), seed, probes, lp[probes], lm[probes], olp, olm) >= 0.99
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name", ["lstm270m", "lstm1b"])
+def test_bf16_large_full_launch_sampled_rows(name):
+    """270M / 1.1B exactly as benchmarked (all probes, batch 1024, T = 10);
+    the oracle evaluates probes 0 and 1 on batch rows 0..31, compared per row
+    (each row's forward is independent of the others), plus the slice losses'
+    sign agreement and the estimate cosine over those probes."""
+    cfg = W.CONFIGS[name]
+    spec = spec_of(cfg)
+    theta = W.init_theta(cfg)
+    tok, tgt = W.batch_for(cfg, step=0)
+    seed = W.step_seed(0)
+    with zo.Context.for_config(cfg) as ctx:
+        lp, lm, rows = gpu_losses(ctx, theta, seed, cfg.n_pert, cfg.eps, tok, tgt, rows=True)
+    assert np.all(np.isfinite(lp)) and np.all(np.isfinite(lm))
+    sl = np.arange(32)
+    probes = [0, 1]
+    olp, olm, orp, orm = O.probe_losses(theta, spec, seed, cfg.n_pert, cfg.eps, tok, tgt,
+                                        probes=probes, rows=sl, return_rows=True)
+    del theta
+    assert np.allclose(rows[probes, 0][:, sl], orp, rtol=1e-2)
+    assert np.allclose(rows[probes, 1][:, sl], orm, rtol=1e-2)
+    cnt = (tgt[sl] >= 0).sum()
+    glp = rows[probes, 0][:, sl].sum(axis=1) / cnt
+    glm = rows[probes, 1][:, sl].sum(axis=1) / cnt
+    assert np.allclose(glp, olp, rtol=1e-2) and np.allclose(glm, olm, rtol=1e-2)
+    assert sign_agreement(glp, glm, olp, olm) >= 0.95
+    assert estimate_cosine(spec, seed, probes, glp, glm, olp, olm) >= 0.99
+    # the full-batch losses are the means of the row sums
+    n_all = (tgt >= 0).sum()
+    assert np.allclose(lp, rows[:, 0].sum(axis=1) / n_all, rtol=1e-5)
+    assert np.allclose(lm, rows[:, 1].sum(axis=1) / n_all, rtol=1e-5)

@@ -52,6 +52,11 @@ struct CellArgs {
   int first;       // t == 0: c_{-1} = 0
   float* raw;      // optional [P][Bmax][4H] pre-activations (then c, h are not written)
   unsigned* err;
+  int gstride;     // rows between the four B boxes (H for the cell, BN/4 for the loss)
+  // cross-entropy epilogue (MODE 1)
+  int V, T, t;
+  const int32_t* targets;  // [B][T]
+  float* rowloss;          // [P][Bmax], accumulated
 };
 
 // ---------------------------------------------------------------------------
@@ -245,7 +250,7 @@ struct TcCfg {
   static_assert(TMEM_COLS == 128 || TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM columns");
 };
 
-template <int MT, int BN, int STAGES, int ACC>
+template <int MT, int BN, int STAGES, int ACC, int MODE>
 __global__ void __launch_bounds__(kTcThreads, 1)
     cell_tc_kernel(const __grid_constant__ CUtensorMap mapA0, const __grid_constant__ CUtensorMap mapA1,
                    const __grid_constant__ CUtensorMap mapW, const CellArgs a, int P) {
@@ -330,7 +335,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           }
 #pragma unroll
           for (int g = 0; g < 4; ++g)
-            tma_load_2d(sb + g * C::U * 128, &mapW, full_bar(s), kk, g * a.H + tc.n * C::U);
+            tma_load_2d(sb + g * C::U * 128, &mapW, full_bar(s), kk, g * a.gstride + tc.n * C::U);
         }
       }
       if (!ok) {
@@ -391,8 +396,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
   } else if (warp < 2 + kGenWarps) {
     // ------------------------------------------------------------ perturbation
-    const int gt = threadIdx.x - 64;  // 0..kGenThreads-1
+    // BN >= kGenThreads: RPT rows per thread, all 8 chunks of each row;
+    // BN <  kGenThreads: TPR threads share a row, CPT chunks each
     constexpr int RPT = (BN + kGenThreads - 1) / kGenThreads;
+    constexpr int TPR = BN >= kGenThreads ? 1 : kGenThreads / BN;
+    constexpr int CPT = 8 / TPR;
+    const int gt = (threadIdx.x - 64) % (BN < kGenThreads ? BN : kGenThreads);
+    const int c0 = ((threadIdx.x - 64) / (BN < kGenThreads ? BN : kGenThreads)) * CPT;
     const float epsf = a.eps;
     const __nv_bfloat16 eb = __float2bfloat16_rn(epsf);
     const uint32_t eps_bits = (uint32_t)(*reinterpret_cast<const uint16_t*>(&eb));
@@ -421,7 +431,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const int r = gt + rr * kGenThreads;
           if (r < BN) {
             const int g = r / C::U, u = r % C::U;
-            const int64_t R = (int64_t)g * a.H + (int64_t)tc.n * C::U + u;
+            const int64_t R = (int64_t)g * a.gstride + (int64_t)tc.n * C::U + u;
             const int64_t j0 = a.offW + R * a.Ktot + (int64_t)kb * 64;
             const int64_t q = j0 >> 7;
             if (q != cq[rr]) {
@@ -433,7 +443,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const uint32_t whi = upper ? cw[rr].w : cw[rr].y;
             uint8_t* row = tileB + r * 128;
 #pragma unroll
-            for (int c16 = 0; c16 < 8; ++c16) {
+            for (int cc = 0; cc < CPT; ++cc) {
+              const int c16 = c0 + cc;
               uint4* p = reinterpret_cast<uint4*>(row + ((c16 ^ (r & 7)) << 4));
               uint4 v = *p;
               const uint32_t w = (c16 < 4 ? wlo : whi) >> (4 * (c16 & 3));
@@ -466,6 +477,43 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       tc_fence_after();
       const float* bias = a.small_p + tc.ps * a.sstride + a.soffb;
+      if constexpr (MODE == 1) {
+        // logits of one row live in one TMEM lane: softmax cross-entropy per row
+        for (int mt = 0; mt < MT; ++mt) {
+          const int b = tc.m * 128 * MT + mt * 128 + rloc;
+          uint32_t z[BN];
+#pragma unroll
+          for (int q = 0; q < BN / 16; ++q) {
+            uint32_t (&zq)[16] = *reinterpret_cast<uint32_t(*)[16]>(z + 16 * q);
+            tmem_ld16(tmem_base + ((uint32_t)(quad * 32) << 16) + ab * C::COLS + mt * BN + 16 * q,
+                      zq);
+          }
+          tmem_wait_ld();
+          if (b < a.B) {
+            int tg = a.targets[(int64_t)b * a.T + a.t];
+            if (tg >= a.V || tg < -1) {
+              latch(a.err, kErrBounds);
+              tg = -1;
+            }
+            if (tg >= 0) {
+              float m = -INFINITY, zt = 0.f;
+#pragma unroll
+              for (int v = 0; v < BN; ++v)
+                if (v < a.V) {
+                  const float zv = __uint_as_float(z[v]) + __ldg(bias + v);
+                  z[v] = __float_as_uint(zv);
+                  m = fmaxf(m, zv);
+                  if (v == tg) zt = zv;
+                }
+              float sum = 0.f;
+#pragma unroll
+              for (int v = 0; v < BN; ++v)
+                if (v < a.V) sum += expf(__uint_as_float(z[v]) - m);
+              a.rowloss[(int64_t)tc.ps * a.Bmax + b] += m + logf(sum) - zt;
+            }
+          }
+        }
+      } else
       for (int mt = 0; mt < MT; ++mt) {
         const int b = tc.m * 128 * MT + mt * 128 + rloc;
         const int64_t rowoff = ((int64_t)tc.ps * a.Bmax + b) * a.H;
@@ -604,11 +652,6 @@ bool map_w(CUtensorMap* m, void* base, int64_t Ktot, int64_t rows, int box_rows)
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Tile configuration.  Large K: 256 rows x 256 gate rows (all 512 TMEM
-// columns, epilogue not overlapped but amortised over K).  Small K: 128 x 256
-// with two accumulators so the epilogue of one tile overlaps the next.
-constexpr int kBN = 256;
-
 }  // namespace
 
 bool make_cell_maps(zo_ctx* c) {
@@ -623,22 +666,23 @@ bool make_cell_maps(zo_ctx* c) {
       ok = ok && map_act(&c->maps->h[l][par], c->h + ((int64_t)l * 2 + par) * P * B * H, H, B, P);
   for (int l = 0; l < L; ++l) {
     const int64_t Ktot = (l == 0 ? E : H) + H;
-    ok = ok && map_w(&c->maps->w[l], c->shadow + c->seg.off[c->seg.W[l]], Ktot, 4 * H, kBN / 4);
+    ok = ok && map_w(&c->maps->w[l], c->shadow + c->seg.off[c->seg.W[l]], Ktot, 4 * H, 64);
   }
+  ok = ok && map_w(&c->maps->wout, c->shadow + c->seg.off[c->seg.Wout], H, s.vocab, 16);
   return ok;
 }
 
-template <int MT, int BN, int STAGES, int ACC>
+template <int MT, int BN, int STAGES, int ACC, int MODE>
 static cudaError_t launch_cfg(const CUtensorMap& A0, const CUtensorMap& A1, const CUtensorMap& Wm,
                               CellArgs a, int P, int sms, cudaStream_t st) {
   using C = TcCfg<MT, BN, STAGES, ACC>;
   a.m_tiles = (a.B + 128 * MT - 1) / (128 * MT);
-  a.n_tiles = a.H / C::U;
+  a.n_tiles = MODE == 0 ? a.H / C::U : 1;
   a.tiles = (int64_t)P * a.m_tiles * a.n_tiles;
-  cudaFuncSetAttribute(cell_tc_kernel<MT, BN, STAGES, ACC>,
+  cudaFuncSetAttribute(cell_tc_kernel<MT, BN, STAGES, ACC, MODE>,
                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   const int64_t grid = a.tiles < sms ? a.tiles : sms;
-  cell_tc_kernel<MT, BN, STAGES, ACC><<<(int)grid, kTcThreads, C::SMEM, st>>>(A0, A1, Wm, a, P);
+  cell_tc_kernel<MT, BN, STAGES, ACC, MODE><<<(int)grid, kTcThreads, C::SMEM, st>>>(A0, A1, Wm, a, P);
   count_launch();
   return cudaGetLastError();
 }
@@ -670,12 +714,58 @@ cudaError_t launch_cell_tc(const zo_ctx* ctx, int layer, int t, int B, int nprob
   a.first = t == 0;
   a.raw = raw_out;
   a.err = ctx->err;
+  a.V = s.vocab;
+  a.T = 0;
+  a.t = t;
+  a.targets = nullptr;
+  a.rowloss = nullptr;
   const CellMaps& m = *ctx->maps;
   const CUtensorMap& A0 = layer == 0 ? m.x : m.h[layer - 1][t & 1];
   const CUtensorMap& A1 = m.h[layer][(t + 1) & 1];
-  if (a.Ktot >= 4096)
-    return launch_cfg<2, kBN, 3, 1>(A0, A1, m.w[layer], a, P, ctx->sm_count, st);
-  return launch_cfg<1, kBN, 4, 2>(A0, A1, m.w[layer], a, P, ctx->sm_count, st);
+  a.gstride = H;
+  // 256 batch rows x 256 gate rows per tile (all 512 TMEM columns): the
+  // fastest shape measured for every model size here (K from 1280 to 16384)
+  return launch_cfg<2, 256, 3, 1, 0>(A0, A1, m.w[layer], a, P, ctx->sm_count, st);
+}
+
+// Output projection + softmax cross-entropy for step t on the same
+// tensor-core mainloop: A = h_top[t] (bf16), B = bf16(W_out) +- eps P formed
+// in shared memory (V <= 64 rows, the rest zero), logits of a row in one TMEM
+// lane; rowloss[ps][b] += logsumexp(z_b) - z_b[target].
+cudaError_t launch_loss_tc(const zo_ctx* ctx, const int32_t* targets, int t, int B, int T,
+                           int nprobe, int probe0, uint64_t seed, float eps, cudaStream_t st) {
+  const zo_model_spec& s = ctx->spec;
+  const int H = s.hidden, L = s.layers;
+  const int P = 2 * nprobe;
+  CellArgs a;
+  a.K0 = H;
+  a.H = H;
+  a.Ktot = H;
+  a.nk = H / 64;
+  a.B = B;
+  a.Bmax = s.max_batch;
+  a.group = 8;
+  a.seed = seed;
+  a.probe0 = probe0;
+  a.eps = eps;
+  a.offW = ctx->seg.off[ctx->seg.Wout];
+  a.small_p = ctx->small_p;
+  a.sstride = ctx->small.stride;
+  a.soffb = ctx->small.bout;
+  a.cst = nullptr;
+  a.hout = nullptr;
+  a.first = 0;
+  a.raw = nullptr;
+  a.err = ctx->err;
+  a.gstride = 16;
+  a.V = s.vocab;
+  a.T = T;
+  a.t = t;
+  a.targets = targets;
+  a.rowloss = ctx->rowloss;
+  const CellMaps& m = *ctx->maps;
+  const CUtensorMap& A0 = m.h[L - 1][t & 1];
+  return launch_cfg<2, 64, 4, 2, 1>(A0, A0, m.wout, a, P, ctx->sm_count, st);
 }
 
 }  // namespace zo

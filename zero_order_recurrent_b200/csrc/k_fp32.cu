@@ -32,7 +32,7 @@ struct Fp32Args {
   unsigned* err;
 };
 
-constexpr int kFpThreads = 512;
+constexpr int kFpThreads = 256;
 
 // Signed perturbation +-eps for element j from the shared sign words.
 __device__ __forceinline__ float pert(const uint32_t* sw, int64_t j, float eps) {
@@ -140,7 +140,7 @@ __device__ void perturbed_gemv(const Fp32Args& a, const uint32_t* sw, int64_t j0
 }
 
 template <int BB, bool VEC>
-__global__ void __launch_bounds__(kFpThreads, 1) fp32_forward_kernel(const Fp32Args a) {
+__global__ void __launch_bounds__(kFpThreads, BB <= 2 ? 4 : 2) fp32_forward_kernel(const Fp32Args a) {
   extern __shared__ __align__(16) float sm[];
   const int ci = blockIdx.x;
   const uint32_t probe = (uint32_t)(a.probe0 + ci);
@@ -241,6 +241,9 @@ template <int BB, bool VEC>
 static cudaError_t launch_fp32_bb(const Fp32Args& a, int nprobe, size_t smem, cudaStream_t st) {
   cudaFuncSetAttribute(fp32_forward_kernel<BB, VEC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                        (int)smem);
+  // ask for the largest shared-memory carveout so several CTAs share an SM
+  cudaFuncSetAttribute(fp32_forward_kernel<BB, VEC>,
+                       cudaFuncAttributePreferredSharedMemoryCarveout, 100);
   int threads = 4 * a.H * 8 / 4;  // 8 lanes per row, 4 rows per warp
   threads = ((threads + 31) / 32) * 32;
   if (threads > kFpThreads) threads = kFpThreads;

@@ -1,7 +1,6 @@
 // Small kernels of the perturbed forward: perturbed copies of the small
-// segments, the embedding gather that builds the first layer's input, the
-// output projection with softmax cross-entropy, and the final per-probe loss
-// reduction.  "Central-difference random-vector gradient estimation evaluates
+// segments, the embedding gather that builds the first layer's input, and the
+// final per-probe loss reduction.  "Central-difference random-vector gradient estimation evaluates
 // complete recurrent forwards at perturbed weights" (alex-wiki, "Method").
 #include "zo_common.cuh"
 #include "zo_internal.h"
@@ -136,108 +135,6 @@ cudaError_t launch_gather_x(const zo_ctx* ctx, const int32_t* tokens, int t, int
   gather_x_kernel<<<(int)grid, 256, 0, st>>>(ctx->small_p, ctx->small.stride, ctx->small.E,
                                              tokens, t, B, T, ctx->spec.max_batch, E,
                                              ctx->spec.vocab, P, ctx->x, ctx->err);
-  count_launch();
-  return cudaGetLastError();
-}
-
-// ---------------------------------------------------------------------------
-// Output projection + softmax cross-entropy for one timestep (bf16 path).
-// Per probe-sign ps: logits[b][v] = h[ps][b][:] . Wout_p[ps][v][:] + bout_p[ps][v];
-// rowloss[ps][b] += logsumexp(logits[b]) - logits[b][target] when scored.
-// CTA tile: 64 rows x 64 logits (V <= 64), K chunks of 32, 4x4 per thread.
-// ---------------------------------------------------------------------------
-constexpr int kLossRows = 64;
-constexpr int kLossCols = 64;
-constexpr int kLossK = 32;
-
-__global__ void __launch_bounds__(256) loss_bf16_kernel(
-    const __nv_bfloat16* __restrict__ h, const float* __restrict__ small_p, int64_t stride,
-    int64_t offW, int64_t offb, const int32_t* __restrict__ targets, int t, int B, int T,
-    int Bmax, int H, int V, float* __restrict__ rowloss, unsigned* err) {
-  __shared__ float As[kLossK][kLossRows + 4];
-  __shared__ float Bs[kLossK][kLossCols + 4];
-  __shared__ float logit[kLossRows][kLossCols + 1];
-  const int ps = blockIdx.y;
-  const int r0 = blockIdx.x * kLossRows;
-  const int tid = threadIdx.x;
-  const int tx = tid & 15, ty = tid >> 4;
-  const __nv_bfloat16* hp = h + (int64_t)ps * Bmax * H;
-  const float* W = small_p + ps * stride + offW;
-  float acc[4][4] = {};
-  for (int k0 = 0; k0 < H; k0 += kLossK) {
-    {  // A: 64 rows x 32 k, 8 bf16 per thread
-      const int row = tid >> 2, kk = (tid & 3) * 8;
-      float v[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-      if (r0 + row < B && k0 + kk + 8 <= H) {
-        const uint4 raw = *reinterpret_cast<const uint4*>(hp + (int64_t)(r0 + row) * H + k0 + kk);
-        const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(&raw);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) v[i] = __bfloat162float(e[i]);
-      } else if (r0 + row < B) {
-        for (int i = 0; i < 8; ++i)
-          if (k0 + kk + i < H) v[i] = __bfloat162float(hp[(int64_t)(r0 + row) * H + k0 + kk + i]);
-      }
-#pragma unroll
-      for (int i = 0; i < 8; ++i) As[kk + i][row] = v[i];
-    }
-    {  // B: 64 logits x 32 k
-      const int col = tid >> 2, kk = (tid & 3) * 8;
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-        Bs[kk + i][col] = (col < V && k0 + kk + i < H) ? W[(int64_t)col * H + k0 + kk + i] : 0.f;
-    }
-    __syncthreads();
-#pragma unroll 8
-    for (int k = 0; k < kLossK; ++k) {
-      float a[4], b[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) a[i] = As[k][ty * 4 + i];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) b[j] = Bs[k][tx * 4 + j];
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
-    }
-    __syncthreads();
-  }
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) logit[ty * 4 + i][tx * 4 + j] = acc[i][j];
-  __syncthreads();
-  if (tid < kLossRows) {
-    const int b = r0 + tid;
-    if (b < B) {
-      int tg = targets[(int64_t)b * T + t];
-      if (tg >= V || tg < -1) {
-        latch(err, kErrBounds);
-        tg = -1;
-      }
-      if (tg >= 0) {
-        const float* bo = small_p + ps * stride + offb;
-        float m = -INFINITY;
-        for (int v = 0; v < V; ++v) m = fmaxf(m, logit[tid][v] + bo[v]);
-        float s = 0.f;
-        for (int v = 0; v < V; ++v) s += expf(logit[tid][v] + bo[v] - m);
-        const float lse = m + logf(s);
-        rowloss[(int64_t)ps * Bmax + b] += lse - (logit[tid][tg] + bo[tg]);
-      }
-    }
-  }
-}
-
-cudaError_t launch_loss_bf16(const zo_ctx* ctx, const int32_t* targets, int t, int B, int T,
-                             int nprobe, cudaStream_t st) {
-  const int L = ctx->spec.layers, H = ctx->spec.hidden;
-  const int P = 2 * nprobe;
-  const int Bmax = ctx->spec.max_batch;
-  const __nv_bfloat16* htop =
-      ctx->h + ((int64_t)(L - 1) * 2 + (t & 1)) * (int64_t)(2 * ctx->chunk) * Bmax * H;
-  dim3 grid((B + kLossRows - 1) / kLossRows, P);
-  loss_bf16_kernel<<<grid, 256, 0, st>>>(htop, ctx->small_p, ctx->small.stride, ctx->small.Wout,
-                                         ctx->small.bout, targets, t, B, T, Bmax, H,
-                                         ctx->spec.vocab, ctx->rowloss, ctx->err);
   count_launch();
   return cudaGetLastError();
 }

@@ -313,8 +313,9 @@ int zo_probe_losses_ex(zo_ctx* ctx, const float* theta, uint64_t seed, int32_t n
           return launch_cell_tc(ctx, l, t, B, np, p0, seed, eps, nullptr, st);
         }));
       }
-      ZO_CUDA(timed(ctx, st, ZO_KIND_LOSS, 2.0 * P * B * Hh * Vv, P * B * Hh * 2.0,
-                    [&] { return launch_loss_bf16(ctx, targets, t, B, T, np, st); }));
+      ZO_CUDA(timed(ctx, st, ZO_KIND_LOSS, 2.0 * P * B * Hh * Vv, P * B * Hh * 2.0, [&] {
+        return launch_loss_tc(ctx, targets, t, B, T, np, p0, seed, eps, st);
+      }));
     }
     ZO_CUDA(timed(ctx, st, ZO_KIND_OTHER, 0.0, 0.0, [&] {
       return launch_reduce_losses(ctx, targets, B, T, p0, np, loss_plus, loss_minus, row_loss, st);

@@ -36,7 +36,8 @@ struct SmallLayout {
 struct CellMaps {
   alignas(64) CUtensorMap x;                    // x_t            [P][B][E]  bf16
   alignas(64) CUtensorMap h[kMaxLayersHost][2];  // h_l (parity)   [P][B][H]  bf16
-  alignas(64) CUtensorMap w[kMaxLayersHost];     // W_l shadow     [4H][in+H] bf16
+  alignas(64) CUtensorMap w[kMaxLayersHost];     // W_l shadow     [4H][in+H] bf16, 64-row box
+  alignas(64) CUtensorMap wout;                  // W_out shadow   [V][H] bf16, 16-row box
 };
 
 }  // namespace zo
@@ -107,8 +108,8 @@ cudaError_t launch_perturb_small(const zo_ctx* ctx, const float* theta, uint64_t
                                  int nprobe, float eps, cudaStream_t st);
 cudaError_t launch_gather_x(const zo_ctx* ctx, const int32_t* tokens, int t, int B, int T,
                             int nprobe, cudaStream_t st);
-cudaError_t launch_loss_bf16(const zo_ctx* ctx, const int32_t* targets, int t, int B, int T,
-                             int nprobe, cudaStream_t st);
+cudaError_t launch_loss_tc(const zo_ctx* ctx, const int32_t* targets, int t, int B, int T,
+                           int nprobe, int probe0, uint64_t seed, float eps, cudaStream_t st);
 cudaError_t launch_cell_tc(const zo_ctx* ctx, int layer, int t, int B, int nprobe, int probe0,
                            uint64_t seed, float eps, float* raw_out, cudaStream_t st);
 bool make_cell_maps(zo_ctx* ctx);
