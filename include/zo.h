@@ -188,6 +188,33 @@ ZO_API int zo_profile(zo_ctx* ctx, int32_t enable);
 ZO_API int zo_profile_read(zo_ctx* ctx, int32_t kind, int64_t* launches, double* total_ms,
                            double* total_flops, double* total_bytes);
 
+/* zo_probe_losses for a ZO_DTYPE_FP32 model without a context and without
+ * allocating anything.  The paper has no counterpart: this exists for callers
+ * that cannot call cudaMalloc at the point where they need the losses - code
+ * running under a memory manager that owns the whole device heap, or a
+ * latency-critical loop that must not take cudaMalloc's implicit device
+ * synchronisation.  Arguments are those of zo_probe_losses (spec replaces the
+ * context; its max_batch, max_seq and chunk fields are ignored).  Every probe
+ * is evaluated in one pass; the per-row loss sums (2 x n_pert x batch floats)
+ * live in a fixed device array of ZO_STATIC_SCRATCH_FLOATS floats that every
+ * GPU loading the library keeps until exit.  Larger requests return
+ * ZO_ERR_INVALID_ARG before anything is launched; models whose fp32 forward
+ * does not fit one CTA's shared memory return ZO_ERR_UNSUPPORTED.
+ * The first call on a device resolves that array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.  All calls share the array and it keeps the last
+ * call's contents: calls that overlap on the GPU (two streams, or two host
+ * threads) race and must be serialised by the caller.  Device-detected input
+ * errors are not reported here (tokens are clamped, out-of-range targets are
+ * not scored): validate tokens and targets beforehand.  No cudaMalloc,
+ * cudaFree or allocating library routine is called.  Async on `stream`. */
+#define ZO_STATIC_SCRATCH_FLOATS 65536
+ZO_API int zo_probe_losses_static(const zo_model_spec* spec, const float* theta_dev,
+                                  uint64_t step_seed, int32_t n_pert, float eps,
+                                  const int32_t* tokens_dev, const int32_t* targets_dev,
+                                  int32_t batch, int32_t seq, float* loss_plus_dev,
+                                  float* loss_minus_dev, void* stream);
+
 /* Human-readable name of a status code (static string). */
 ZO_API const char* zo_status_string(int status);
 

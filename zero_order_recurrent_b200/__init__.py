@@ -31,8 +31,9 @@ EXPORTS = (
     "zo_create", "zo_destroy", "zo_param_layout", "zo_workspace_info", "zo_probe_losses",
     "zo_probe_losses_ex", "zo_coeffs", "zo_update", "zo_invalidate_shadow", "zo_step_host",
     "zo_sync_status", "zo_sign_words", "zo_status_string", "zo_kernel_launches",
-    "zo_debug_cell_preact", "zo_profile", "zo_profile_read",
+    "zo_debug_cell_preact", "zo_profile", "zo_profile_read", "zo_probe_losses_static",
 )
+ZO_STATIC_SCRATCH_FLOATS = 65536
 ZO_KIND_CELL, ZO_KIND_LOSS, ZO_KIND_UPDATE, ZO_KIND_OTHER = 0, 1, 2, 3
 
 
@@ -78,6 +79,8 @@ def load_library(path: str = LIB_PATH):
         "zo_kernel_launches": ([], I64),
         "zo_debug_cell_preact": ([P, P, U64, I32, I32, F, P, I32, I32, P, P], ctypes.c_int),
         "zo_profile": ([P, I32], ctypes.c_int),
+        "zo_probe_losses_static": ([ctypes.POINTER(ModelSpec), P, U64, I32, F, P, P, I32, I32, P, P,
+                                    P], ctypes.c_int),
         "zo_profile_read": ([P, I32, ctypes.POINTER(I64), ctypes.POINTER(ctypes.c_double),
                              ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double)],
                             ctypes.c_int),
@@ -236,6 +239,16 @@ def zo_profile_read(ctx, kind: int):
     _check(load_library().zo_profile_read(ctx.handle, kind, ctypes.byref(n), ctypes.byref(ms),
                                           ctypes.byref(fl), ctypes.byref(by)), "zo_profile_read")
     return n.value, ms.value, fl.value, by.value
+
+
+def zo_probe_losses_static(spec: ModelSpec, theta, step_seed, n_pert, eps, tokens, targets,
+                           loss_plus, loss_minus, stream=None) -> int:
+    """Context-free fp32 probe losses that allocate no device memory (see
+    include/zo.h).  Returns the status code instead of raising."""
+    B, T = tokens.shape
+    return load_library().zo_probe_losses_static(
+        ctypes.byref(spec), _ptr(theta), ctypes.c_uint64(step_seed), n_pert, eps, _ptr(tokens),
+        _ptr(targets), B, T, _ptr(loss_plus), _ptr(loss_minus), _stream(stream))
 
 
 def zo_kernel_launches() -> int:

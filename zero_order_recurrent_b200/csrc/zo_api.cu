@@ -116,6 +116,11 @@ bool bf16_shape_ok(const zo_model_spec& s) {
 
 }  // namespace
 
+namespace zo {
+// The flat parameter layout of a spec (the same one zo_create builds).
+void layout_of(const zo_model_spec& sp, Segments& s) { build_segments(sp, s); }
+}  // namespace zo
+
 extern "C" {
 
 const char* zo_status_string(int st) {

@@ -113,5 +113,7 @@ cudaError_t launch_loss_tc(const zo_ctx* ctx, const int32_t* targets, int t, int
 cudaError_t launch_cell_tc(const zo_ctx* ctx, int layer, int t, int B, int nprobe, int probe0,
                            uint64_t seed, float eps, float* raw_out, cudaStream_t st);
 bool make_cell_maps(zo_ctx* ctx);
+void layout_of(const zo_model_spec& sp, Segments& s);
+size_t fp32_smem_bytes(const zo_model_spec& s, int bb, int64_t d_pad);
 
 }  // namespace zo
