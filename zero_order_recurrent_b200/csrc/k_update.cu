@@ -114,15 +114,32 @@ struct UpdateArgs {
   unsigned* err;
 };
 
+// Packed fp32x2 add (sm_100): two independent round-to-nearest sums.
+__device__ __forceinline__ float2 add_f32x2(float2 a, float2 b) {
+  unsigned long long ar = *reinterpret_cast<unsigned long long*>(&a);
+  unsigned long long br = *reinterpret_cast<unsigned long long*>(&b);
+  unsigned long long r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(ar), "l"(br));
+  return *reinterpret_cast<float2*>(&r);
+}
+
+// PP > 0: compile-time probes per pass (n <= PP, unused slots carry c = 0,
+// whose +-0 terms leave every sum unchanged), coefficients in registers and
+// S = 512 / PP blocks per span.  PP == 0: runtime n, S and passes.
+template <int PP>
 __global__ void __launch_bounds__(kUpdWarps * 32) update_kernel(const UpdateArgs a) {
+  constexpr int SC = PP > 0 ? (kUpdSlots / PP < 32 ? kUpdSlots / PP : 32) : 1;
   extern __shared__ uint4 dyn[];
-  float* negc = reinterpret_cast<float*>(dyn);             // [n], padded to 4
-  uint4* words_all = dyn + (a.n + 3) / 4;                   // [warps][kUpdSlots]
+  const int ncap = PP > 0 ? PP : a.n;
+  float* negc = reinterpret_cast<float*>(dyn);             // [ncap], padded to 4
+  uint4* words_all = dyn + (ncap + 3) / 4;                  // [warps][kUpdSlots]
+  const int S = PP > 0 ? SC : a.S;
+  float4* stage_all = reinterpret_cast<float4*>(words_all + kUpdWarps * kUpdSlots);  // [warps][S*32]
   __shared__ int bad;
   if (threadIdx.x == 0) bad = 0;
   __syncthreads();
-  for (int i = threadIdx.x; i < a.n; i += blockDim.x) {
-    const float c = a.coeffs[i];
+  for (int i = threadIdx.x; i < ncap; i += blockDim.x) {
+    const float c = i < a.n ? a.coeffs[i] : 0.f;
     if (!isfinite(c)) bad = 1;
     negc[i] = -c;
   }
@@ -135,13 +152,18 @@ __global__ void __launch_bounds__(kUpdWarps * 32) update_kernel(const UpdateArgs
   const int warp = threadIdx.x >> 5;
   uint4* words = words_all + warp * kUpdSlots;
   const uint32_t* words32 = reinterpret_cast<const uint32_t*>(words);
-  const int S = a.S;
+  float4* stage = stage_all + warp * S * 32;
   const int64_t nspan = (a.nblk + S - 1) / S;
   const int64_t gw = blockIdx.x * (int64_t)kUpdWarps + warp;
   const int64_t nw = (int64_t)gridDim.x * kUpdWarps;
   const int widx = lane >> 3;
   const int sh = 2 * (lane & 7);
   const float4* th4 = reinterpret_cast<const float4*>(a.theta);
+  float ncr[PP > 0 ? PP : 1];
+  if constexpr (PP > 0) {
+#pragma unroll
+    for (int i = 0; i < PP; ++i) ncr[i] = negc[i];
+  }
 
   for (int64_t span = gw; span < nspan; span += nw) {
     const int64_t q0 = span * S;
@@ -149,40 +171,67 @@ __global__ void __launch_bounds__(kUpdWarps * 32) update_kernel(const UpdateArgs
     // segment of the span's first block; segments start on block boundaries
     int seg = 0;
     while (seg + 1 < a.nseg && q0 * 128 >= a.seg_off[seg + 1]) ++seg;
-    for (int p0 = 0; p0 < a.n; p0 += a.pmax) {
-      const int np = min(a.pmax, a.n - p0);
-      const bool last_pass = p0 + a.pmax >= a.n;
+    const int pmax = PP > 0 ? PP : a.pmax;
+    for (int p0 = 0; p0 < a.n; p0 += pmax) {
+      const int np = min(pmax, a.n - p0);
+      const bool last_pass = p0 + pmax >= a.n;
+      // start the span's theta loads so that they land during the sign phase
+      // (a later pass re-reads what this lane stored in the previous one)
+      if (p0 > 0) __threadfence_block();
+      for (int it = 0; it < nq; ++it) {
+        const uint32_t dst = (uint32_t)__cvta_generic_to_shared(stage + it * 32 + lane);
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst),
+                     "l"(th4 + (q0 + it) * 32 + lane)
+                     : "memory");
+      }
+      asm volatile("cp.async.commit_group;" ::: "memory");
       const int pairs = np * S;
 #pragma unroll 4
       for (int t = lane; t < pairs; t += 32) {
         const int i = t / S, b = t - i * S;
         if (b < nq) words[t] = sign_block(a.seed, (uint32_t)(p0 + i), (uint64_t)(q0 + b));
       }
+      asm volatile("cp.async.wait_all;" ::: "memory");
       __syncwarp();
       int sg = seg;
-      float4 nxt = th4[q0 * 32 + lane];
       for (int it = 0; it < nq; ++it) {
         const int64_t q = q0 + it;
-        const float4 th = nxt;
-        if (it + 1 < nq) nxt = th4[(q + 1) * 32 + lane];
+        const float4 th = stage[it * 32 + lane];
         double acc0 = th.x, acc1 = th.y, acc2 = th.z, acc3 = th.w;
         const uint32_t* wcol = words32 + it * 4 + widx;
-        for (int g = 0; g < np; g += 8) {
-          float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-          const int ge = min(g + 8, np);
-#pragma unroll 8
-          for (int i = g; i < ge; ++i) {
-            const float nc = negc[p0 + i];
-            const uint32_t w = wcol[i * S * 4] >> sh;
-            s0 += flip_sign(nc, w << 31);
-            s1 += flip_sign(nc, w << 15);
-            s2 += flip_sign(nc, w << 30);
-            s3 += flip_sign(nc, w << 14);
+        if constexpr (PP > 0) {
+#pragma unroll
+          for (int g = 0; g < PP; g += 8) {
+            float2 s01 = make_float2(0.f, 0.f), s23 = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int i = g; i < g + 8; ++i) {
+              const uint32_t w = wcol[i * SC * 4] >> sh;
+              s01 = add_f32x2(s01, make_float2(flip_sign(ncr[i], w << 31), flip_sign(ncr[i], w << 15)));
+              s23 = add_f32x2(s23, make_float2(flip_sign(ncr[i], w << 30), flip_sign(ncr[i], w << 14)));
+            }
+            acc0 += s01.x;
+            acc1 += s01.y;
+            acc2 += s23.x;
+            acc3 += s23.y;
           }
-          acc0 += s0;
-          acc1 += s1;
-          acc2 += s2;
-          acc3 += s3;
+        } else {
+          for (int g = 0; g < np; g += 8) {
+            float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+            const int ge = min(g + 8, np);
+#pragma unroll 8
+            for (int i = g; i < ge; ++i) {
+              const float nc = negc[p0 + i];
+              const uint32_t w = wcol[i * S * 4] >> sh;
+              s0 += flip_sign(nc, w << 31);
+              s1 += flip_sign(nc, w << 15);
+              s2 += flip_sign(nc, w << 30);
+              s3 += flip_sign(nc, w << 14);
+            }
+            acc0 += s0;
+            acc1 += s1;
+            acc2 += s2;
+            acc3 += s3;
+          }
         }
         while (sg + 1 < a.nseg && q * 128 >= a.seg_off[sg + 1]) ++sg;
         const int64_t j = q * 128 + 4 * lane;
@@ -207,6 +256,25 @@ __global__ void __launch_bounds__(kUpdWarps * 32) update_kernel(const UpdateArgs
   }
 }
 
+template <int PP>
+static cudaError_t launch_update_pp(const UpdateArgs& a, int sm_count, cudaStream_t st) {
+  const int ncap = PP > 0 ? PP : a.n;
+  const size_t smem = sizeof(uint4) * ((ncap + 3) / 4 + (size_t)kUpdWarps * kUpdSlots +
+                                      (size_t)kUpdWarps * a.S * 32);
+  cudaFuncSetAttribute(update_kernel<PP>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaFuncSetAttribute(update_kernel<PP>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+  const int64_t nspan = (a.nblk + a.S - 1) / a.S;
+  int64_t grid = (nspan + kUpdWarps - 1) / kUpdWarps;
+  int per_sm = (int)((200 * 1024) / smem);
+  if (per_sm < 1) per_sm = 1;
+  if (per_sm > 8) per_sm = 8;
+  const int64_t cap = (int64_t)sm_count * per_sm;
+  if (grid > cap) grid = cap;
+  update_kernel<PP><<<(int)grid, kUpdWarps * 32, smem, st>>>(a);
+  count_launch();
+  return cudaGetLastError();
+}
+
 cudaError_t launch_update(const zo_ctx* ctx, float* theta, uint64_t seed, int n,
                           const float* coeffs, __nv_bfloat16* shadow, cudaStream_t st) {
   UpdateArgs a;
@@ -222,26 +290,27 @@ cudaError_t launch_update(const zo_ctx* ctx, float* theta, uint64_t seed, int n,
     a.seg_end[s] = ctx->seg.off[s] + ctx->seg.numel[s];
   }
   a.err = ctx->err;
+  const int64_t want = (int64_t)ctx->sm_count * 16;   // spans that fill the GPU
+  // compile-time probe counts for large models
+  const int pp = n <= 16 ? 16 : n <= 32 ? 32 : n <= 64 ? 64 : 0;
+  if (pp) {
+    const int S = kUpdSlots / pp < 32 ? kUpdSlots / pp : 32;
+    if ((a.nblk + S - 1) / S >= want) {
+      a.S = S;
+      a.pmax = pp;
+      if (pp == 16) return launch_update_pp<16>(a, ctx->sm_count, st);
+      if (pp == 32) return launch_update_pp<32>(a, ctx->sm_count, st);
+      return launch_update_pp<64>(a, ctx->sm_count, st);
+    }
+  }
   // blocks per span: all probes in one pass if possible, and enough spans
   // to give every SM 16 warps of work
   int S = 32;
   while (S > 1 && S * n > kUpdSlots) S /= 2;
-  const int64_t want = (int64_t)ctx->sm_count * 16;
   while (S > 1 && (a.nblk + S - 1) / S < want) S /= 2;
   a.S = S;
   a.pmax = kUpdSlots / S < n ? kUpdSlots / S : n;
-  const size_t smem = sizeof(uint4) * ((n + 3) / 4 + (size_t)kUpdWarps * kUpdSlots);
-  cudaFuncSetAttribute(update_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  const int64_t nspan = (a.nblk + S - 1) / S;
-  int64_t grid = (nspan + kUpdWarps - 1) / kUpdWarps;
-  int per_sm = (int)((200 * 1024) / smem);
-  if (per_sm < 1) per_sm = 1;
-  if (per_sm > 8) per_sm = 8;
-  const int64_t cap = (int64_t)ctx->sm_count * per_sm;
-  if (grid > cap) grid = cap;
-  update_kernel<<<(int)grid, kUpdWarps * 32, smem, st>>>(a);
-  count_launch();
-  return cudaGetLastError();
+  return launch_update_pp<0>(a, ctx->sm_count, st);
 }
 
 }  // namespace zo
