@@ -72,44 +72,57 @@ def batches(cfg, n, rank):
 
 
 class ClockSampler:
-    def __init__(self, gpu_index, path):
-        self.path = path
+    """nvidia-smi samples (every 50 ms) with host timestamps; `summary` keeps
+    the samples that fall inside a wall-clock window."""
+
+    def __init__(self, gpu_index):
+        import tempfile
         self.proc = None
+        self.path = os.path.join(tempfile.mkdtemp(prefix="zo_clocks_"), "clocks.csv")
         try:
-            self.f = open(path, "w")
+            self.f = open(self.path, "w")
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={gpu_index}", f"--query-gpu={CLOCK_QUERY}", "--format=csv,noheader",
-                 "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+                ["nvidia-smi", f"--id={gpu_index}", f"--query-gpu=timestamp,{CLOCK_QUERY}",
+                 "--format=csv,noheader", "-lms", "50"], stdout=self.f, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
 
     def stop(self):
         if self.proc is None:
-            return None
+            return
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
         except Exception:
             self.proc.kill()
         self.f.close()
-        sm, mx, reasons = [], [], set()
+
+    def summary(self, t0, t1):
+        if self.proc is None:
+            return None
+        import datetime
+        rows = []
         for line in open(self.path):
             f = [x.strip() for x in line.split(",")]
-            if len(f) < 9:
+            if len(f) < 10:
                 continue
             try:
-                sm.append(float(f[1].split()[0]))
-                mx.append(float(f[2].split()[0]))
+                ts = datetime.datetime.strptime(f[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                sm, mx = float(f[2].split()[0]), float(f[3].split()[0])
             except ValueError:
                 continue
             names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-            for nm, v in zip(names, f[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(nm)
-        if not sm:
+            rs = {nm for nm, v in zip(names, f[6:10]) if v.lower().startswith("active")}
+            rows.append((ts, sm, mx, rs))
+        if not rows:
             return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+        inside = [r for r in rows if t0 <= r[0] <= t1]
+        if not inside:   # window shorter than the sampling period: nearest sample
+            inside = [min(rows, key=lambda r: abs(r[0] - 0.5 * (t0 + t1)))]
+        reasons = set().union(*[r[3] for r in inside])
+        return {"sm_mhz": statistics.median(r[1] for r in inside),
+                "sm_max_mhz": max(r[2] for r in inside), "reasons": sorted(reasons),
+                "samples": len(inside)}
 
 
 def run_ours(args, cfg):
@@ -146,6 +159,7 @@ def run_ours(args, cfg):
         zo.cdrge_step(ctx, theta, W.step_seed(k, run_seed=rank), n, eps, eta, toks[k], tgts[k],
                       lp, lm, coef)
 
+    sampler = ClockSampler(local)
     for k in range(Wm):
         step(k)
     torch.cuda.synchronize()
@@ -155,9 +169,8 @@ def run_ours(args, cfg):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    sampler = ClockSampler(local, os.path.join(ROOT, "gpurun_out", f"clocks_rank{rank}.csv")) \
-        if os.path.isdir(os.path.join(ROOT, "gpurun_out")) or True else None
     launches0 = zo.zo_kernel_launches()
+    t_start = time.time()
     zo.zo_profile(ctx, True)
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
     for k in range(K):
@@ -166,9 +179,11 @@ def run_ours(args, cfg):
         step(Wm + k)
         ev[k][1].record(st)
     torch.cuda.synchronize()
+    t_end = time.time()
     zo.zo_profile(ctx, False)
     launches = zo.zo_kernel_launches() - launches0
-    clocks = sampler.stop() if sampler else None
+    sampler.stop()
+    clocks = sampler.summary(t_start, t_end)
     s = zo.zo_sync_status(ctx)
     if s != zo.ZO_OK:
         raise RuntimeError(f"timed steps failed: {zo.status_string(s)}")
@@ -213,6 +228,23 @@ def run_ours(args, cfg):
             "rank": rank, "world": world}
 
 
+def captured_traffic(cfg):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu
+    summary (profiles/traffic.json), or None when there is none or the
+    kernel's source changed since the capture."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    e = json.load(open(p)).get(cfg.name)
+    if not e:
+        return None
+    src = os.path.join(ROOT, e["source"])
+    if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest()[:16] != e["sha256_16"]:
+        return None
+    return e["bytes_per_launch"]
+
+
 def roofline_for(cfg, kinds, clocks, pk):
     n_cell, ms_cell, fl_cell, _ = kinds["cell"]
     if cfg.dtype == "bf16":
@@ -220,7 +252,7 @@ def roofline_for(cfg, kinds, clocks, pk):
         peak = pk["bf16_tflops_sustained"]
         return {"bound": "tensor", "kernel": "cell_tc_kernel (tcgen05 perturbed LSTM cell)",
                 "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
-                "frac": round(achieved / peak, 4), "traffic": None,
+                "frac": round(achieved / peak, 4), "traffic": captured_traffic(cfg),
                 "peak_source": f"{pk['source']} bf16 dense, sustained",
                 "launches": n_cell, "avg_launch_ms": round(ms_cell / max(n_cell, 1), 4)}
     achieved = fl_cell / (ms_cell / 1e3) / 1e12
@@ -228,7 +260,7 @@ def roofline_for(cfg, kinds, clocks, pk):
     peak = fp32_alu_peak_tflops(mhz)
     return {"bound": "alu", "kernel": "fp32_forward_kernel (persistent perturbed LSTM forward)",
             "achieved": round(achieved, 3), "peak": round(peak, 2), "unit": "TFLOP/s",
-            "frac": round(achieved / peak, 4), "traffic": None,
+            "frac": round(achieved / peak, 4), "traffic": captured_traffic(cfg),
             "peak_source": f"fp32 FMA: 148 SMs x 128 lanes x 2 x {mhz:.0f} MHz",
             "launches": n_cell, "avg_launch_ms": round(ms_cell / max(n_cell, 1), 4)}
 
