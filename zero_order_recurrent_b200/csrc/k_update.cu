@@ -124,17 +124,23 @@ __device__ __forceinline__ float2 add_f32x2(float2 a, float2 b) {
 }
 
 // PP > 0: compile-time probes per pass (n <= PP, unused slots carry c = 0,
-// whose +-0 terms leave every sum unchanged), coefficients in registers and
-// S = 512 / PP blocks per span.  PP == 0: runtime n, S and passes.
+// whose +-0 terms leave every sum unchanged), coefficients in registers,
+// S = 128 / PP blocks per span (PP * S = 128 sign blocks: four Philox calls
+// per lane) and theta staged in two buffers: the next span's loads are in
+// flight while the current span is applied.  Small spans keep the shared
+// memory per warp at ~10 KB, so 20 warps share an SM.
+// PP == 0: runtime n, S and passes, one staging buffer.
 template <int PP>
 __global__ void __launch_bounds__(kUpdWarps * 32) update_kernel(const UpdateArgs a) {
-  constexpr int SC = PP > 0 ? (kUpdSlots / PP < 32 ? kUpdSlots / PP : 32) : 1;
+  constexpr int SC = PP > 0 ? (128 / PP < 32 ? 128 / PP : 32) : 1;
+  constexpr int WSLOTS = PP > 0 ? PP * SC : kUpdSlots;   // sign-word slots per warp
+  constexpr int NBUF = PP > 0 ? 2 : 1;
   extern __shared__ uint4 dyn[];
   const int ncap = PP > 0 ? PP : a.n;
   float* negc = reinterpret_cast<float*>(dyn);             // [ncap], padded to 4
-  uint4* words_all = dyn + (ncap + 3) / 4;                  // [warps][kUpdSlots]
+  uint4* words_all = dyn + (ncap + 3) / 4;                  // [warps][WSLOTS]
   const int S = PP > 0 ? SC : a.S;
-  float4* stage_all = reinterpret_cast<float4*>(words_all + kUpdWarps * kUpdSlots);  // [warps][S*32]
+  float4* stage_all = reinterpret_cast<float4*>(words_all + kUpdWarps * WSLOTS);  // [warps][NBUF][S*32]
   __shared__ int bad;
   if (threadIdx.x == 0) bad = 0;
   __syncthreads();
@@ -150,9 +156,9 @@ __global__ void __launch_bounds__(kUpdWarps * 32) update_kernel(const UpdateArgs
   }
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
-  uint4* words = words_all + warp * kUpdSlots;
+  uint4* words = words_all + warp * WSLOTS;
   const uint32_t* words32 = reinterpret_cast<const uint32_t*>(words);
-  float4* stage = stage_all + warp * S * 32;
+  float4* stage = stage_all + warp * NBUF * S * 32;
   const int64_t nspan = (a.nblk + S - 1) / S;
   const int64_t gw = blockIdx.x * (int64_t)kUpdWarps + warp;
   const int64_t nw = (int64_t)gridDim.x * kUpdWarps;
@@ -165,9 +171,24 @@ __global__ void __launch_bounds__(kUpdWarps * 32) update_kernel(const UpdateArgs
     for (int i = 0; i < PP; ++i) ncr[i] = negc[i];
   }
 
-  for (int64_t span = gw; span < nspan; span += nw) {
+  auto issue = [&](int64_t sp, float4* dstbuf) {
+    const int64_t qq = sp * S;
+    const int nn = (int)min((int64_t)S, a.nblk - qq);
+    for (int it = 0; it < nn; ++it) {
+      const uint32_t dst = (uint32_t)__cvta_generic_to_shared(dstbuf + it * 32 + lane);
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst),
+                   "l"(th4 + (qq + it) * 32 + lane)
+                   : "memory");
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+  int buf = 0;
+  if (PP > 0 && gw < nspan) issue(gw, stage);
+
+  for (int64_t span = gw; span < nspan; span += nw, buf ^= (NBUF - 1)) {
     const int64_t q0 = span * S;
     const int nq = (int)min((int64_t)S, a.nblk - q0);
+    float4* cur = stage + buf * S * 32;
     // segment of the span's first block; segments start on block boundaries
     int seg = 0;
     while (seg + 1 < a.nseg && q0 * 128 >= a.seg_off[seg + 1]) ++seg;
@@ -175,28 +196,31 @@ __global__ void __launch_bounds__(kUpdWarps * 32) update_kernel(const UpdateArgs
     for (int p0 = 0; p0 < a.n; p0 += pmax) {
       const int np = min(pmax, a.n - p0);
       const bool last_pass = p0 + pmax >= a.n;
-      // start the span's theta loads so that they land during the sign phase
-      // (a later pass re-reads what this lane stored in the previous one)
-      if (p0 > 0) __threadfence_block();
-      for (int it = 0; it < nq; ++it) {
-        const uint32_t dst = (uint32_t)__cvta_generic_to_shared(stage + it * 32 + lane);
-        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst),
-                     "l"(th4 + (q0 + it) * 32 + lane)
-                     : "memory");
+      if (PP == 0) {
+        // theta loads land during the sign phase (a later pass re-reads what
+        // this lane stored in the previous one)
+        if (p0 > 0) __threadfence_block();
+        issue(span, cur);
       }
-      asm volatile("cp.async.commit_group;" ::: "memory");
       const int pairs = np * S;
 #pragma unroll 4
       for (int t = lane; t < pairs; t += 32) {
         const int i = t / S, b = t - i * S;
         if (b < nq) words[t] = sign_block(a.seed, (uint32_t)(p0 + i), (uint64_t)(q0 + b));
       }
-      asm volatile("cp.async.wait_all;" ::: "memory");
+      if (PP > 0) {
+        // next span's theta into the other buffer, then wait for this span's
+        if (span + nw < nspan) issue(span + nw, stage + (buf ^ 1) * S * 32);
+        else asm volatile("cp.async.commit_group;" ::: "memory");
+        asm volatile("cp.async.wait_group 1;" ::: "memory");
+      } else {
+        asm volatile("cp.async.wait_all;" ::: "memory");
+      }
       __syncwarp();
       int sg = seg;
       for (int it = 0; it < nq; ++it) {
         const int64_t q = q0 + it;
-        const float4 th = stage[it * 32 + lane];
+        const float4 th = cur[it * 32 + lane];
         double acc0 = th.x, acc1 = th.y, acc2 = th.z, acc3 = th.w;
         const uint32_t* wcol = words32 + it * 4 + widx;
         if constexpr (PP > 0) {
@@ -259,13 +283,14 @@ __global__ void __launch_bounds__(kUpdWarps * 32) update_kernel(const UpdateArgs
 template <int PP>
 static cudaError_t launch_update_pp(const UpdateArgs& a, int sm_count, cudaStream_t st) {
   const int ncap = PP > 0 ? PP : a.n;
-  const size_t smem = sizeof(uint4) * ((ncap + 3) / 4 + (size_t)kUpdWarps * kUpdSlots +
-                                      (size_t)kUpdWarps * a.S * 32);
+  const size_t wslots = PP > 0 ? (size_t)PP * a.S : (size_t)kUpdSlots;
+  const size_t smem = sizeof(uint4) * ((ncap + 3) / 4 + (size_t)kUpdWarps * wslots +
+                                      (size_t)kUpdWarps * (PP > 0 ? 2 : 1) * a.S * 32);
   cudaFuncSetAttribute(update_kernel<PP>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   cudaFuncSetAttribute(update_kernel<PP>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
   const int64_t nspan = (a.nblk + a.S - 1) / a.S;
   int64_t grid = (nspan + kUpdWarps - 1) / kUpdWarps;
-  int per_sm = (int)((200 * 1024) / smem);
+  int per_sm = (int)((220 * 1024) / smem);
   if (per_sm < 1) per_sm = 1;
   if (per_sm > 8) per_sm = 8;
   const int64_t cap = (int64_t)sm_count * per_sm;
@@ -294,7 +319,7 @@ cudaError_t launch_update(const zo_ctx* ctx, float* theta, uint64_t seed, int n,
   // compile-time probe counts for large models
   const int pp = n <= 16 ? 16 : n <= 32 ? 32 : n <= 64 ? 64 : 0;
   if (pp) {
-    const int S = kUpdSlots / pp < 32 ? kUpdSlots / pp : 32;
+    const int S = 128 / pp < 32 ? 128 / pp : 32;
     if ((a.nblk + S - 1) / S >= want) {
       a.S = S;
       a.pmax = pp;
