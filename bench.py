@@ -7,11 +7,13 @@ A step is zo_probe_losses + zo_coeffs + zo_update over one synthetic batch of
 the named workload (default "overfit", the single-batch overfitting setting;
 also tiny, charlm, lstm270m, lstm1b).  `value` is CD-RGE steps/s of the whole
 job (device time, inputs resident in HBM, L2 flushed before every step and
-the flush not timed).  `e2e` is the same metric through zo_step_host with the
-step's tokens/targets copied from pinned host memory and L+/L- read back.
-With N > 1 (torchrun) every rank runs an independent replica on its own batch
-(weak scaling; no collective in the data path) and the time is the max over
-ranks.  `--impl reference` times the fp64 CPU oracle instead (rank 0 only).
+the flush not timed).  `e2e` is the same metric with the step's
+tokens/targets copied from pinned host memory and L+/L- read back every step
+(zo_step_host on one GPU).  With N > 1 (torchrun) the n_pert probes of each
+step are split over the ranks (probe_parallel: each rank evaluates its probe
+slice, the 2 n_pert scalar losses are all-gathered over NCCL, every rank
+applies the same update): strong scaling, time = max over ranks.
+`--impl reference` times the fp64 CPU oracle instead (rank 0 only).
 """
 from __future__ import annotations
 
@@ -145,7 +147,7 @@ def run_ours(args, cfg):
     theta = torch.from_numpy(theta_h).to(dev)
     del theta_h
     K, Wm = args.steps, args.warmup
-    bl = batches(cfg, Wm + K, rank)
+    bl = batches(cfg, Wm + K, 0)
     toks = [torch.from_numpy(t).to(dev) for t, _ in bl]
     tgts = [torch.from_numpy(g).to(dev) for _, g in bl]
     lp = torch.empty(n, device=dev)
@@ -156,8 +158,11 @@ def run_ours(args, cfg):
     st = torch.cuda.current_stream()
 
     def step(k):
-        zo.cdrge_step(ctx, theta, W.step_seed(k, run_seed=rank), n, eps, eta, toks[k], tgts[k],
-                      lp, lm, coef)
+        if world > 1:
+            from zero_order_recurrent_b200.probe_parallel import cdrge_step_sharded
+            cdrge_step_sharded(ctx, theta, W.step_seed(k), n, eps, eta, toks[k], tgts[k], coef)
+        else:
+            zo.cdrge_step(ctx, theta, W.step_seed(k), n, eps, eta, toks[k], tgts[k], lp, lm, coef)
 
     sampler = ClockSampler(local)
     for k in range(Wm):
@@ -209,15 +214,25 @@ def run_ours(args, cfg):
         torch.cuda.synchronize()
         t0 = time.perf_counter()
         for k in range(Ke):
-            zo.zo_step_host(ctx, theta, W.step_seed(Wm + K + k, run_seed=rank), n, eps, eta, ht[k % len(ht)],
-                            hg[k % len(hg)], hp, hm)
+            seed = W.step_seed(Wm + K + k)
+            if world > 1:
+                from zero_order_recurrent_b200.probe_parallel import cdrge_step_sharded
+                tk = ht[k % len(ht)].to(dev, non_blocking=True)
+                tg = hg[k % len(hg)].to(dev, non_blocking=True)
+                glp, glm = cdrge_step_sharded(ctx, theta, seed, n, eps, eta, tk, tg, coef)
+                hp.copy_(glp, non_blocking=True)
+                hm.copy_(glm, non_blocking=True)
+                torch.cuda.current_stream().synchronize()
+            else:
+                zo.zo_step_host(ctx, theta, seed, n, eps, eta, ht[k % len(ht)], hg[k % len(hg)],
+                                hp, hm)
         torch.cuda.synchronize()
         e_ms = (time.perf_counter() - t0) * 1e3
         if world > 1:
             t = torch.tensor([e_ms], device=dev)
             dist.all_reduce(t, op=dist.ReduceOp.MAX)
             e_ms = float(t.item())
-        e2e = {"value": world * Ke / (e_ms / 1e3), "unit": "steps/s",
+        e2e = {"value": Ke / (e_ms / 1e3), "unit": "steps/s",
                "h2d_bytes_per_step": 2 * cfg.batch * cfg.seq * 4, "d2h_bytes_per_step": 2 * n * 4,
                "steps": Ke}
     ctx.close()
@@ -319,8 +334,9 @@ def main():
     config = {"workload": f"{cfg.name}: {cfg.layers}-layer LSTM V={cfg.vocab} E={cfg.embed} H={cfg.hidden}, "
                           f"batch {cfg.batch} x seq {cfg.seq}, n_pert={cfg.n_pert}, eps=eta={cfg.eps}",
               "params": int(W.segments(cfg.vocab, cfg.embed, cfg.hidden, cfg.layers)[1]),
-              "global_batch": cfg.batch * world, "seq_len": cfg.seq, "n_pert": cfg.n_pert,
-              "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+              "global_batch": cfg.batch, "seq_len": cfg.seq, "n_pert": cfg.n_pert,
+              "parallelism": (f"probe-parallel x{world} (NCCL all-gather of the 2 n_pert losses)"
+                              if world > 1 else "single GPU"),
               "l2": "flushed (256 MB write) before every timed step, flush untimed",
               "tokens": "seeded synthetic (workloads module)"}
     dtype = "bf16" if cfg.dtype == "bf16" else "f32"
@@ -333,7 +349,7 @@ def main():
         print(json.dumps({"metric": METRIC, "impl": "reference", "value": v, "unit": "steps/s",
                           "perturbed_tokens_per_s": v * tokens_per_step, "n_gpus": world,
                           "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 / v,
-                          "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                          "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
                           "dtype": "f64", "data": "synthetic", "config": config,
                           "cpu_baseline": cb,
                           "e2e": {"value": v, "unit": "steps/s", "h2d_bytes_per_step": 0,
@@ -346,11 +362,11 @@ def main():
     if rank != 0:
         return
     pk = peaks()
-    value = world * args.steps / (r["ms"] / 1e3)
+    value = args.steps / (r["ms"] / 1e3)
     out = {"metric": METRIC, "value": value, "unit": "steps/s",
            "perturbed_tokens_per_s": value * tokens_per_step, "n_gpus": world, "steps": args.steps,
            "warmup": args.warmup, "ms_per_step": r["ms"] / args.steps, "higher_is_better": True,
-           "scaling": "weak", "vs_baseline": None, "dtype": dtype, "data": "synthetic",
+           "scaling": "strong", "vs_baseline": None, "dtype": dtype, "data": "synthetic",
            "config": config, "roofline": roofline_for(cfg, r["kinds"], r["clocks"], pk)}
     nu, msu, _, byu = r["kinds"]["update"]
     if nu:

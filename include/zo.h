@@ -129,6 +129,20 @@ ZO_API int zo_probe_losses_ex(zo_ctx* ctx, const float* theta_dev, uint64_t step
                        int32_t batch, int32_t seq, float* loss_plus_dev, float* loss_minus_dev,
                        float* row_loss_dev, void* stream);
 
+/* Losses of the probe slice probe_begin .. probe_begin + n_probes - 1 only,
+ * written to loss_plus_dev[i], loss_minus_dev[i] (fp32 [n_probes]); probe
+ * probe_begin + i is exactly probe probe_begin + i of zo_probe_losses.  This
+ * is the unit of the probe-parallel scheme of the pith.science review ("What
+ * carries the argument": workers each compute a few perturbed losses and only
+ * scalar losses travel): each process evaluates one slice and the slices'
+ * losses are gathered before zo_coeffs.  Other arguments and behaviour as
+ * zo_probe_losses.  Async on `stream`. */
+ZO_API int zo_probe_losses_slice(zo_ctx* ctx, const float* theta_dev, uint64_t step_seed,
+                                 int32_t probe_begin, int32_t n_probes, float eps,
+                                 const int32_t* tokens_dev, const int32_t* targets_dev,
+                                 int32_t batch, int32_t seq, float* loss_plus_dev,
+                                 float* loss_minus_dev, void* stream);
+
 /* Coefficients c_i = eta (L+_i - L-_i) / (2 eps n_pert) (alex-wiki "Method";
  * eta = eps gives the review's 1/(2 n_pert) factor).  fp32 [n_pert] in and
  * out, device.  A non-finite input latches ZO_ERR_NONFINITE and writes NaN

@@ -364,3 +364,26 @@ def test_bf16_large_full_launch_sampled_rows(name):
     n_all = (tgt >= 0).sum()
     assert np.allclose(lp, rows[:, 0].sum(axis=1) / n_all, rtol=1e-5)
     assert np.allclose(lm, rows[:, 1].sum(axis=1) / n_all, rtol=1e-5)
+
+
+@pytest.mark.parametrize("name,slices", [("tiny", [(0, 3), (3, 5)]), ("charlm", [(0, 2), (5, 1), (62, 2)])])
+def test_probe_slices_match_full_call(name, slices):
+    """zo_probe_losses_slice(probe_begin, n) returns entries probe_begin ..
+    probe_begin + n - 1 of zo_probe_losses, bit for bit (the unit of the
+    probe-parallel scheme)."""
+    cfg = W.CONFIGS[name]
+    theta = dev(W.init_theta(cfg))
+    B = min(cfg.batch, 128)
+    tok, tgt = W.batch_for(cfg)
+    tok, tgt = dev(tok[:B]), dev(tgt[:B])
+    n = cfg.n_pert
+    with zo.Context.for_config(cfg, max_batch=B, chunk=8 if cfg.dtype == "bf16" else None) as ctx:
+        lp = torch.empty(n, device="cuda")
+        lm = torch.empty(n, device="cuda")
+        zo.zo_probe_losses(ctx, theta, 9, n, cfg.eps, tok, tgt, lp, lm)
+        for b0, c in slices:
+            sp = torch.empty(c, device="cuda")
+            sm = torch.empty(c, device="cuda")
+            zo.zo_probe_losses_slice(ctx, theta, 9, b0, c, cfg.eps, tok, tgt, sp, sm)
+            assert zo.zo_sync_status(ctx) == zo.ZO_OK
+            assert torch.equal(sp, lp[b0:b0 + c]) and torch.equal(sm, lm[b0:b0 + c])

@@ -32,6 +32,7 @@ EXPORTS = (
     "zo_probe_losses_ex", "zo_coeffs", "zo_update", "zo_invalidate_shadow", "zo_step_host",
     "zo_sync_status", "zo_sign_words", "zo_status_string", "zo_kernel_launches",
     "zo_debug_cell_preact", "zo_profile", "zo_profile_read", "zo_probe_losses_static",
+    "zo_probe_losses_slice",
 )
 ZO_STATIC_SCRATCH_FLOATS = 65536
 ZO_KIND_CELL, ZO_KIND_LOSS, ZO_KIND_UPDATE, ZO_KIND_OTHER = 0, 1, 2, 3
@@ -79,6 +80,7 @@ def load_library(path: str = LIB_PATH):
         "zo_kernel_launches": ([], I64),
         "zo_debug_cell_preact": ([P, P, U64, I32, I32, F, P, I32, I32, P, P], ctypes.c_int),
         "zo_profile": ([P, I32], ctypes.c_int),
+        "zo_probe_losses_slice": ([P, P, U64, I32, I32, F, P, P, I32, I32, P, P, P], ctypes.c_int),
         "zo_probe_losses_static": ([ctypes.POINTER(ModelSpec), P, U64, I32, F, P, P, I32, I32, P, P,
                                     P], ctypes.c_int),
         "zo_profile_read": ([P, I32, ctypes.POINTER(I64), ctypes.POINTER(ctypes.c_double),
@@ -179,6 +181,15 @@ def zo_probe_losses(ctx, theta, step_seed, n_pert, eps, tokens, targets, loss_pl
         ctx.handle, _ptr(theta), ctypes.c_uint64(step_seed), n_pert, eps, _ptr(tokens),
         _ptr(targets), B, T, _ptr(loss_plus), _ptr(loss_minus), _ptr(row_loss), _stream(stream)),
         "zo_probe_losses")
+
+
+def zo_probe_losses_slice(ctx, theta, step_seed, probe_begin, n_probes, eps, tokens, targets,
+                          loss_plus, loss_minus, stream=None):
+    B, T = tokens.shape
+    _check(load_library().zo_probe_losses_slice(
+        ctx.handle, _ptr(theta), ctypes.c_uint64(step_seed), probe_begin, n_probes, eps,
+        _ptr(tokens), _ptr(targets), B, T, _ptr(loss_plus), _ptr(loss_minus), _stream(stream)),
+        "zo_probe_losses_slice")
 
 
 def zo_coeffs(ctx, loss_plus, loss_minus, n_pert, eps, eta, coeffs, stream=None):

@@ -3,6 +3,7 @@
 // the update driver.  Every kernel runs on the caller's stream; nothing here
 // synchronises except zo_create, zo_destroy, zo_step_host and zo_sync_status.
 #include <math.h>
+#include <stdint.h>
 #include <stdio.h>
 #include <stdlib.h>
 #include <string.h>
@@ -270,11 +271,17 @@ int zo_invalidate_shadow(zo_ctx* ctx) {
   return ZO_OK;
 }
 
-int zo_probe_losses_ex(zo_ctx* ctx, const float* theta, uint64_t seed, int32_t n_pert, float eps,
-                       const int32_t* tokens, const int32_t* targets, int32_t batch, int32_t seq,
-                       float* loss_plus, float* loss_minus, float* row_loss, void* stream) {
+// Losses of probes probe_begin .. probe_begin + n_pert - 1 (the probes' signs
+// use their global index), written to loss_plus[i], loss_minus[i] for
+// i < n_pert.
+static int probe_losses_range(zo_ctx* ctx, const float* theta, uint64_t seed, int32_t probe_begin,
+                              int32_t n_pert, float eps, const int32_t* tokens,
+                              const int32_t* targets, int32_t batch, int32_t seq, float* loss_plus,
+                              float* loss_minus, float* row_loss, void* stream) {
   if (!ctx || !theta || !tokens || !targets || !loss_plus || !loss_minus) return ZO_ERR_INVALID_ARG;
-  if (n_pert < 1 || !(eps > 0.f) || !isfinite(eps)) return ZO_ERR_INVALID_ARG;
+  if (n_pert < 1 || probe_begin < 0 || (int64_t)probe_begin + n_pert > INT32_MAX ||
+      !(eps > 0.f) || !isfinite(eps))
+    return ZO_ERR_INVALID_ARG;
   if (batch < 1 || batch > ctx->spec.max_batch || seq < 1 || seq > ctx->spec.max_seq)
     return ZO_ERR_INVALID_ARG;
   cudaStream_t st = S(stream);
@@ -287,7 +294,8 @@ int zo_probe_losses_ex(zo_ctx* ctx, const float* theta, uint64_t seed, int32_t n
       const int np = n_pert - p0 < ctx->chunk ? n_pert - p0 : ctx->chunk;
       const double fl = 2.0 * 2 * np * (double)B * T * fwd_macs;
       ZO_CUDA(timed(ctx, st, ZO_KIND_CELL, fl, 0.0, [&] {
-        return launch_fp32_forward(ctx, theta, seed, p0, np, eps, tokens, targets, B, T, st);
+        return launch_fp32_forward(ctx, theta, seed, probe_begin + p0, np, eps, tokens, targets, B,
+                                   T, st);
       }));
       ZO_CUDA(timed(ctx, st, ZO_KIND_OTHER, 0.0, 0.0, [&] {
         return launch_reduce_losses(ctx, targets, B, T, p0, np, loss_plus, loss_minus, row_loss, st);
@@ -306,7 +314,7 @@ int zo_probe_losses_ex(zo_ctx* ctx, const float* theta, uint64_t seed, int32_t n
     const int np = n_pert - p0 < ctx->chunk ? n_pert - p0 : ctx->chunk;
     const double P = 2.0 * np;
     ZO_CUDA(timed(ctx, st, ZO_KIND_OTHER, 0.0, 0.0,
-                  [&] { return launch_perturb_small(ctx, theta, seed, p0, np, eps, st); }));
+                  [&] { return launch_perturb_small(ctx, theta, seed, probe_begin + p0, np, eps, st); }));
     ZO_CUDA(cudaMemsetAsync(ctx->rowloss, 0, sizeof(float) * 2 * np * ctx->spec.max_batch, st));
     for (int t = 0; t < T; ++t) {
       ZO_CUDA(timed(ctx, st, ZO_KIND_OTHER, 0.0, P * B * Ee * 2.0,
@@ -315,11 +323,11 @@ int zo_probe_losses_ex(zo_ctx* ctx, const float* theta, uint64_t seed, int32_t n
         const double Krun = (double)(l == 0 ? Ee : Hh) + (t == 0 ? 0.0 : (double)Hh);
         const double fl = 2.0 * P * B * Krun * 4.0 * Hh;
         ZO_CUDA(timed(ctx, st, ZO_KIND_CELL, fl, 0.0, [&] {
-          return launch_cell_tc(ctx, l, t, B, np, p0, seed, eps, nullptr, st);
+          return launch_cell_tc(ctx, l, t, B, np, probe_begin + p0, seed, eps, nullptr, st);
         }));
       }
       ZO_CUDA(timed(ctx, st, ZO_KIND_LOSS, 2.0 * P * B * Hh * Vv, P * B * Hh * 2.0, [&] {
-        return launch_loss_tc(ctx, targets, t, B, T, np, p0, seed, eps, st);
+        return launch_loss_tc(ctx, targets, t, B, T, np, probe_begin + p0, seed, eps, st);
       }));
     }
     ZO_CUDA(timed(ctx, st, ZO_KIND_OTHER, 0.0, 0.0, [&] {
@@ -327,6 +335,21 @@ int zo_probe_losses_ex(zo_ctx* ctx, const float* theta, uint64_t seed, int32_t n
     }));
   }
   return ZO_OK;
+}
+
+int zo_probe_losses_ex(zo_ctx* ctx, const float* theta, uint64_t seed, int32_t n_pert, float eps,
+                       const int32_t* tokens, const int32_t* targets, int32_t batch, int32_t seq,
+                       float* loss_plus, float* loss_minus, float* row_loss, void* stream) {
+  return probe_losses_range(ctx, theta, seed, 0, n_pert, eps, tokens, targets, batch, seq,
+                            loss_plus, loss_minus, row_loss, stream);
+}
+
+int zo_probe_losses_slice(zo_ctx* ctx, const float* theta, uint64_t seed, int32_t probe_begin,
+                          int32_t n_probes, float eps, const int32_t* tokens,
+                          const int32_t* targets, int32_t batch, int32_t seq, float* loss_plus,
+                          float* loss_minus, void* stream) {
+  return probe_losses_range(ctx, theta, seed, probe_begin, n_probes, eps, tokens, targets, batch,
+                            seq, loss_plus, loss_minus, nullptr, stream);
 }
 
 int zo_probe_losses(zo_ctx* ctx, const float* theta, uint64_t seed, int32_t n_pert, float eps,
