@@ -387,3 +387,34 @@ def test_probe_slices_match_full_call(name, slices):
             zo.zo_probe_losses_slice(ctx, theta, 9, b0, c, cfg.eps, tok, tgt, sp, sm)
             assert zo.zo_sync_status(ctx) == zo.ZO_OK
             assert torch.equal(sp, lp[b0:b0 + c]) and torch.equal(sm, lm[b0:b0 + c])
+
+
+@pytest.mark.parametrize("V,E,H,L,B,T,n,chunk,frac", [
+    (50, 128, 64, 3, 300, 3, 3, 0, 0.0),    # three layers, E != H, ragged 256-row tiles
+    (64, 64, 128, 2, 257, 2, 5, 2, 0.2),    # V = 64 (all logit columns), 3 chunks (2, 2, 1)
+    (2, 64, 64, 1, 1, 4, 2, 0, 0.0),        # V = 2, a single batch row
+    (33, 64, 64, 2, 128, 1, 4, 0, 0.0),     # T = 1 (no recurrent input at all)
+    (50, 64, 64, 1, 100, 3, 2, 0, 1.0),     # nothing scored: losses 0
+])
+def test_bf16_edge_cases(V, E, H, L, B, T, n, chunk, frac):
+    cfg = W.small_config(vocab=V, embed=E, hidden=H, layers=L, dtype="bf16")
+    theta = W.init_theta(cfg, seed=2)
+    tok, tgt = W.random_batch(B, T, V, seed=5, ignore_frac=frac)
+    seed = W.step_seed(8)
+    with zo.Context(V, E, H, L, "bf16", B, T, chunk) as ctx:
+        lp, lm, rows = gpu_losses(ctx, theta, seed, n, 1e-3, tok, tgt, rows=True)
+    olp, olm, orp, orm = O.probe_losses(theta, (V, E, H, L), seed, n, 1e-3, tok, tgt,
+                                        return_rows=True)
+    if frac == 1.0:
+        assert np.all(lp == 0) and np.all(lm == 0) and np.all(rows == 0)
+        return
+    assert np.allclose(lp, olp, rtol=1e-2) and np.allclose(lm, olm, rtol=1e-2)
+    assert np.allclose(rows[:, 0], orp, rtol=1e-2, atol=1e-3)
+    assert np.allclose(rows[:, 1], orm, rtol=1e-2, atol=1e-3)
+
+
+def test_bf16_shape_limits_are_reported():
+    for V, E, H in ((65, 64, 64), (50, 48, 64), (50, 64, 96)):
+        with pytest.raises(zo.ZOError) as e:
+            zo.Context(V, E, H, 1, "bf16", 8, 2, 1)
+        assert e.value.status == zo.ZO_ERR_UNSUPPORTED
