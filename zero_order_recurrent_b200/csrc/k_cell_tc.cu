@@ -138,6 +138,13 @@ __device__ __forceinline__ void prefetch_map(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
+// Bulk prefetch of [p, p + bytes) into L2 (16-byte aligned, multiple of 16).
+__device__ __forceinline__ void prefetch_l2(const void* p, int bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)),
+               "r"(bytes)
+               : "memory");
+}
+
 __device__ __forceinline__ void fence_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
@@ -471,6 +478,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const TileCoord tc = decode_tile(a, tile, P);
       const int ab = tcount % ACC;
       const uint32_t aph = (tcount / ACC) & 1;
+      if (MODE == 0 && !a.first && !a.raw) {
+        // while this tile's MMAs run, pull its c_{t-1} rows into L2 so the
+        // epilogue's loads hit L2 rather than HBM
+        for (int mt = 0; mt < MT; ++mt) {
+          const int b = tc.m * 128 * MT + mt * 128 + rloc;
+          if (b < a.B)
+            prefetch_l2(a.cst + ((int64_t)tc.ps * a.Bmax + b) * a.H + tc.n * C::U,
+                        C::U * (int)sizeof(float));
+        }
+      }
       if (!mbar_wait(accf_bar(ab), aph, abort_flag, a.err)) {
         ok = false;
         break;
@@ -517,6 +534,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       for (int mt = 0; mt < MT; ++mt) {
         const int b = tc.m * 128 * MT + mt * 128 + rloc;
         const int64_t rowoff = ((int64_t)tc.ps * a.Bmax + b) * a.H;
+        const bool live = b < a.B;
+        const bool need_c = live && !a.first && !a.raw;
+        float4* crow = reinterpret_cast<float4*>(a.cst + rowoff + tc.n * C::U);
+        // c_{t-1} of the next 8-unit chunk is loaded one chunk ahead, so its
+        // latency overlaps this chunk's TMEM load and gate arithmetic
+        float4 cn0 = make_float4(0.f, 0.f, 0.f, 0.f), cn1 = cn0;
+        if (need_c) {
+          cn0 = crow[0];
+          cn1 = crow[1];
+        }
 #pragma unroll 1
         for (int u0 = 0; u0 < C::U; u0 += 8) {
           uint32_t acc[4][8];
@@ -525,8 +552,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             tmem_ld8(tmem_base + ((uint32_t)(quad * 32) << 16) + ab * C::COLS + mt * BN +
                          g * C::U + u0,
                      acc[g]);
+          const float4 cc0 = cn0, cc1 = cn1;
+          if (need_c && u0 + 8 < C::U) {
+            cn0 = crow[(u0 >> 2) + 2];
+            cn1 = crow[(u0 >> 2) + 3];
+          }
           tmem_wait_ld();
-          if (b < a.B) {
+          if (live) {
             const int unit0 = tc.n * C::U + u0;
             float pre[4][8];
 #pragma unroll
@@ -551,21 +583,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                       make_float4(pre[g][4 * q4], pre[g][4 * q4 + 1], pre[g][4 * q4 + 2],
                                   pre[g][4 * q4 + 3]);
             } else {
-              float cprev[8];
-              float4* cp = reinterpret_cast<float4*>(a.cst + rowoff + unit0);
-              if (a.first) {
-#pragma unroll
-                for (int i = 0; i < 8; ++i) cprev[i] = 0.f;
-              } else {
-#pragma unroll
-                for (int q4 = 0; q4 < 2; ++q4) {
-                  const float4 v = cp[q4];
-                  cprev[4 * q4] = v.x;
-                  cprev[4 * q4 + 1] = v.y;
-                  cprev[4 * q4 + 2] = v.z;
-                  cprev[4 * q4 + 3] = v.w;
-                }
-              }
+              const float cprev[8] = {cc0.x, cc0.y, cc0.z, cc0.w, cc1.x, cc1.y, cc1.z, cc1.w};
               float cn[8];
               uint32_t hp[4];
 #pragma unroll
@@ -583,9 +601,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 __nv_bfloat162 pr = __floats2bfloat162_rn(hv[0], hv[1]);
                 hp[i >> 1] = *reinterpret_cast<uint32_t*>(&pr);
               }
-#pragma unroll
-              for (int q4 = 0; q4 < 2; ++q4)
-                cp[q4] = make_float4(cn[4 * q4], cn[4 * q4 + 1], cn[4 * q4 + 2], cn[4 * q4 + 3]);
+              crow[(u0 >> 2)] = make_float4(cn[0], cn[1], cn[2], cn[3]);
+              crow[(u0 >> 2) + 1] = make_float4(cn[4], cn[5], cn[6], cn[7]);
               *reinterpret_cast<uint4*>(a.hout + rowoff + unit0) = make_uint4(hp[0], hp[1], hp[2], hp[3]);
             }
           }
