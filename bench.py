@@ -86,6 +86,9 @@ class ClockSampler:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={gpu_index}", f"--query-gpu=timestamp,{CLOCK_QUERY}",
                  "--format=csv,noheader", "-lms", "50"], stdout=self.f, stderr=subprocess.DEVNULL)
+            t0 = time.time()   # nvidia-smi takes a moment before its first line
+            while time.time() - t0 < 3.0 and os.path.getsize(self.path) == 0:
+                time.sleep(0.05)
         except Exception:
             self.proc = None
 

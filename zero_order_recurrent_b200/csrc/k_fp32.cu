@@ -385,8 +385,13 @@ cudaError_t launch_fp32_forward(const zo_ctx* ctx, const float* theta, uint64_t 
   a.rowloss = ctx->rowloss;
   a.err = ctx->err;
   const bool vec = (a.E % 4 == 0) && (a.H % 4 == 0);
-  return vec ? launch_fp32_vec<true>(a, ctx->fp32_bb, nprobe, ctx->fp32_smem, st)
-             : launch_fp32_vec<false>(a, ctx->fp32_bb, nprobe, ctx->fp32_smem, st);
+  // rows per CTA: the context's maximum, halved while probes x row blocks
+  // leave SMs idle (a CTA's shared memory shrinks with its rows)
+  int bb = ctx->fp32_bb;
+  while (bb > 1 && (int64_t)nprobe * ((B + bb - 1) / bb) < ctx->sm_count) bb /= 2;
+  const size_t smem = fp32_smem_bytes(ctx->spec, bb, s.d_pad);
+  return vec ? launch_fp32_vec<true>(a, bb, nprobe, smem, st)
+             : launch_fp32_vec<false>(a, bb, nprobe, smem, st);
 }
 
 }  // namespace zo
