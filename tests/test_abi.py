@@ -31,6 +31,14 @@ def test_header_declares_the_binding_exports():
     assert declared_functions() == sorted(zo.EXPORTS)
 
 
+def test_header_constants_match_the_binding():
+    src = "".join(open(h).read() for h in glob.glob(os.path.join(INCLUDE, "*.h")))
+    defines = dict(re.findall(r"#define\s+(ZO_[A-Z0-9_]+)\s+(-?\d+)\b", src))
+    assert defines, "no integer constants found in the headers"
+    for name, value in defines.items():
+        assert getattr(zo, name) == int(value), name
+
+
 def test_library_exports_every_declared_symbol(lib):
     for name in declared_functions():
         assert hasattr(lib, name), name

@@ -94,7 +94,12 @@ def _check_update(cfg, n, theta, seed, coeffs, ctx, idx=None):
     return th
 
 
-@pytest.mark.parametrize("name,n", [("tiny", 8), ("overfit", 512), ("overfit", 37)])
+# every probe-group count the update kernel compiles (1, 2, 4, 8, 16 groups of
+# four probes), counts that leave a group partly empty, and several passes
+@pytest.mark.parametrize("name,n", [("tiny", 8), ("tiny", 1), ("tiny", 3), ("overfit", 512),
+                                    ("overfit", 37), ("overfit", 5), ("overfit", 13),
+                                    ("overfit", 16), ("overfit", 29), ("overfit", 32),
+                                    ("overfit", 64), ("overfit", 65), ("overfit", 100)])
 def test_update_matches_oracle(name, n):
     cfg = W.CONFIGS[name]
     theta = W.init_theta(cfg)
@@ -102,6 +107,18 @@ def test_update_matches_oracle(name, n):
     coeffs = np.random.default_rng(n).standard_normal(n) * 1e-3
     with zo.Context.for_config(cfg) as ctx:
         _check_update(cfg, n, theta, seed, coeffs, ctx)
+
+
+def test_update_rejects_too_many_probes():
+    cfg = W.CONFIGS["tiny"]
+    n = zo.ZO_MAX_UPDATE_PROBES + 1
+    th = dev(W.init_theta(cfg))
+    c = torch.zeros(n, device="cuda")
+    with zo.Context.for_config(cfg) as ctx:
+        with pytest.raises(zo.ZOError) as e:
+            zo.zo_update(ctx, th, 1, n, c)
+        assert e.value.status == zo.ZO_ERR_INVALID_ARG
+        assert torch.equal(th, dev(W.init_theta(cfg)))
 
 
 def test_update_bf16_context_sampled_and_shadow():

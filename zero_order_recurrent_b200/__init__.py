@@ -35,6 +35,7 @@ EXPORTS = (
     "zo_probe_losses_slice",
 )
 ZO_STATIC_SCRATCH_FLOATS = 65536
+ZO_MAX_UPDATE_PROBES = 8192
 ZO_KIND_CELL, ZO_KIND_LOSS, ZO_KIND_UPDATE, ZO_KIND_OTHER = 0, 1, 2, 3
 
 

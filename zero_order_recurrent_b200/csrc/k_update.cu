@@ -86,18 +86,25 @@ cudaError_t launch_coeffs(const float* lp, const float* lm, int n, float eps, fl
 }
 
 // ---------------------------------------------------------------------------
-// Update.  One warp handles a span of S consecutive 128-element blocks.  In
-// the sign phase the 32 lanes compute the Philox words of all (probe, block)
-// pairs of the span and park them in shared memory; in the apply phase the
-// warp walks the span block by block, lane L owning the float4 at 4L..4L+3,
-// so every global access is a coalesced 512-byte row.  Probes are summed in
-// fp32 groups of 8 and the groups in fp64, then theta is rounded once.  S is
-// chosen on the host so that all probes fit one pass (S * probes <= 512
-// words per warp) and the spans still fill the GPU; with more probes than
-// that, successive passes re-read theta.
+// Update.  theta'_j = theta_j + sum_i (-c_i) p_ij is evaluated four probes at
+// a time through subset-sum tables: for the probes 4g..4g+3 of group g,
+//   T_g[s] = sum_{r<4} (-c_{4g+r}) (1 - 2 s_r),   s = 4-bit sign pattern,
+// (16 entries, computed in fp64 and rounded once) so one shared-memory lookup
+// replaces four sign applications.  The tables hold 16 consecutive words, one
+// per bank, so a warp's lookups never conflict.
+//
+// One warp handles a span of S consecutive 128-element blocks.  Sign phase:
+// lane t owns one (group, block) pair, computes its four probes' Philox
+// blocks and transposes the bits so that each byte holds one parameter's
+// 4-bit pattern, pre-shifted to a word offset (pattern << 2), and parks them
+// in shared memory.  Apply phase: lane L owns the float4 at 4L..4L+3 of each
+// block (coalesced 512-byte rows) and, per group, takes its four bytes with
+// byte permutes and sums the four table entries per parameter in a pairwise
+// tree.  theta is staged by cp.async in two buffers, so the next span's
+// loads are in flight during this span's work.
 // ---------------------------------------------------------------------------
 constexpr int kUpdWarps = 4;
-constexpr int kUpdSlots = 512;   // uint4 sign-word slots per warp (8 KB)
+constexpr int kPairStride = 17;   // 8-byte units per (group, block) pair: 16 + 1 pad
 
 struct UpdateArgs {
   float* theta;
@@ -105,9 +112,9 @@ struct UpdateArgs {
   const float* coeffs;
   uint64_t seed;
   int n;
+  int ngroups;             // table groups (chunks * NG)
+  int chunks;              // passes of NG groups over each span
   int64_t nblk;            // d_pad / 128
-  int S;                   // blocks per span
-  int pmax;                // probes per pass (pmax * S <= kUpdSlots)
   int nseg;
   int64_t seg_off[kMaxSeg];
   int64_t seg_end[kMaxSeg];
@@ -123,31 +130,61 @@ __device__ __forceinline__ float2 add_f32x2(float2 a, float2 b) {
   return *reinterpret_cast<float2*>(&r);
 }
 
-// PP > 0: compile-time probes per pass (n <= PP, unused slots carry c = 0,
-// whose +-0 terms leave every sum unchanged), coefficients in registers,
-// S = 128 / PP blocks per span (PP * S = 128 sign blocks: four Philox calls
-// per lane) and theta staged in two buffers: the next span's loads are in
-// flight while the current span is applied.  Small spans keep the shared
-// memory per warp at ~10 KB, so 20 warps share an SM.
-// PP == 0: runtime n, S and passes, one staging buffer.
-template <int PP>
-__global__ void __launch_bounds__(kUpdWarps * 32) update_kernel(const UpdateArgs a) {
-  constexpr int SC = PP > 0 ? (128 / PP < 32 ? 128 / PP : 32) : 1;
-  constexpr int WSLOTS = PP > 0 ? PP * SC : kUpdSlots;   // sign-word slots per warp
-  constexpr int NBUF = PP > 0 ? 2 : 1;
-  extern __shared__ uint4 dyn[];
-  const int ncap = PP > 0 ? PP : a.n;
-  float* negc = reinterpret_cast<float*>(dyn);             // [ncap], padded to 4
-  uint4* words_all = dyn + (ncap + 3) / 4;                  // [warps][WSLOTS]
-  const int S = PP > 0 ? SC : a.S;
-  float4* stage_all = reinterpret_cast<float4*>(words_all + kUpdWarps * WSLOTS);  // [warps][NBUF][S*32]
+// Bits of a where m is set, bits of b elsewhere.
+__device__ __forceinline__ uint32_t bit_select(uint32_t m, uint32_t a, uint32_t b) {
+  return (a & m) | (b & ~m);
+}
+
+// Transposes four probes' sign words (A = probe 4g, ..., D = probe 4g+3; bit p
+// = word position p) into eight index words: byte j of W[c] holds, at bits
+// 2..5, the pattern (A,B,C,D)[c + 8j] as bits 0..3.  Two interleaving steps
+// pair up bits and then bit pairs of the four words (nibble u of n_s holds
+// position 4u + (0,2,1,3)[s]); the last step spreads the nibbles to bytes.
+__device__ __forceinline__ void index_bytes(uint32_t A, uint32_t B, uint32_t C, uint32_t D,
+                                            uint32_t (&W)[8]) {
+  const uint32_t m1 = 0x55555555u, m2 = 0x33333333u, m4 = 0x3C3C3C3Cu;
+  const uint32_t abe = bit_select(m1, A, B << 1), abo = bit_select(m1, A >> 1, B);
+  const uint32_t cde = bit_select(m1, C, D << 1), cdo = bit_select(m1, C >> 1, D);
+  const uint32_t n0 = bit_select(m2, abe, cde << 2), n1 = bit_select(m2, abe >> 2, cde);
+  const uint32_t n2 = bit_select(m2, abo, cdo << 2), n3 = bit_select(m2, abo >> 2, cdo);
+  W[0] = (n0 << 2) & m4;
+  W[1] = (n2 << 2) & m4;
+  W[2] = (n1 << 2) & m4;
+  W[3] = (n3 << 2) & m4;
+  W[4] = (n0 >> 2) & m4;
+  W[5] = (n2 >> 2) & m4;
+  W[6] = (n1 >> 2) & m4;
+  W[7] = (n3 >> 2) & m4;
+}
+
+__device__ __forceinline__ float table_at(const float* t, uint32_t byte_off) {
+  return *reinterpret_cast<const float*>(reinterpret_cast<const char*>(t) + byte_off);
+}
+
+// NG groups (4 NG probes) per pass.  MULTI: runtime number of passes, each
+// pass's fp32 tree sum added into an fp64 accumulator (n_pert > 64).
+template <int NG, bool MULTI>
+__global__ void __launch_bounds__(kUpdWarps * 32, 4) update_kernel(const UpdateArgs a) {
+  constexpr int S = NG >= 4 ? 32 / NG : 8;   // blocks per span
+  constexpr int PAIRS = NG * S;              // (group, block) pairs of a pass, <= 32
+  extern __shared__ __align__(16) unsigned char dyn[];
+  float* tab = reinterpret_cast<float*>(dyn);                       // [ngroups][16]
+  uint2* idx_all = reinterpret_cast<uint2*>(dyn + a.ngroups * 64);  // [warps][32][kPairStride]
+  float4* stage_all = reinterpret_cast<float4*>(idx_all + kUpdWarps * 32 * kPairStride);
   __shared__ int bad;
   if (threadIdx.x == 0) bad = 0;
   __syncthreads();
-  for (int i = threadIdx.x; i < ncap; i += blockDim.x) {
-    const float c = i < a.n ? a.coeffs[i] : 0.f;
-    if (!isfinite(c)) bad = 1;
-    negc[i] = -c;
+  for (int e = threadIdx.x; e < a.ngroups * 16; e += blockDim.x) {
+    const int g = e >> 4, s = e & 15;
+    double t = 0.0;
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int i = 4 * g + r;
+      const float c = i < a.n ? a.coeffs[i] : 0.f;
+      if (!isfinite(c)) bad = 1;
+      t += ((s >> r) & 1) ? (double)c : -(double)c;
+    }
+    tab[e] = (float)t;
   }
   __syncthreads();
   if (bad) {
@@ -156,20 +193,19 @@ __global__ void __launch_bounds__(kUpdWarps * 32) update_kernel(const UpdateArgs
   }
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
-  uint4* words = words_all + warp * WSLOTS;
-  const uint32_t* words32 = reinterpret_cast<const uint32_t*>(words);
-  float4* stage = stage_all + warp * NBUF * S * 32;
+  uint2* idxw = idx_all + warp * 32 * kPairStride;
+  float4* stage = stage_all + warp * 2 * S * 32;
   const int64_t nspan = (a.nblk + S - 1) / S;
   const int64_t gw = blockIdx.x * (int64_t)kUpdWarps + warp;
   const int64_t nw = (int64_t)gridDim.x * kUpdWarps;
-  const int widx = lane >> 3;
-  const int sh = 2 * (lane & 7);
   const float4* th4 = reinterpret_cast<const float4*>(a.theta);
-  float ncr[PP > 0 ? PP : 1];
-  if constexpr (PP > 0) {
-#pragma unroll
-    for (int i = 0; i < PP; ++i) ncr[i] = negc[i];
-  }
+  // apply role: word lane>>3, elements 4m..4m+3 (m = lane & 7) at positions
+  // 2m, 2m+16, 2m+1, 2m+17 = bytes (m>>2, m>>2 + 2) of index words 2(m&3), +1
+  const int unit = (lane >> 3) * 4 + (lane & 3);
+  const uint32_t sel_lo = 0x4440u | (uint32_t)((lane & 7) >> 2);
+  const uint32_t sel_hi = sel_lo + 2;
+  // sign role: this lane's (group, block) pair
+  const int pg = lane / S, pb = lane % S;
 
   auto issue = [&](int64_t sp, float4* dstbuf) {
     const int64_t qq = sp * S;
@@ -182,120 +218,141 @@ __global__ void __launch_bounds__(kUpdWarps * 32) update_kernel(const UpdateArgs
     }
     asm volatile("cp.async.commit_group;" ::: "memory");
   };
+  // theta' of block q: pads past the block's segment end keep theta, and the
+  // bf16 shadow gets the same values
+  auto write_out = [&](int64_t q, int& sg, float4 th, float4 o) {
+    while (sg + 1 < a.nseg && q * 128 >= a.seg_off[sg + 1]) ++sg;
+    const int64_t lim = a.seg_end[sg];
+    if (q * 128 + 128 > lim) {
+      const int64_t j = q * 128 + 4 * lane;
+      o.x = j + 0 < lim ? o.x : th.x;
+      o.y = j + 1 < lim ? o.y : th.y;
+      o.z = j + 2 < lim ? o.z : th.z;
+      o.w = j + 3 < lim ? o.w : th.w;
+    }
+    reinterpret_cast<float4*>(a.theta)[q * 32 + lane] = o;
+    if (a.shadow) {
+      __nv_bfloat162 lo = __floats2bfloat162_rn(o.x, o.y);
+      __nv_bfloat162 hi = __floats2bfloat162_rn(o.z, o.w);
+      uint2 pk;
+      pk.x = *reinterpret_cast<uint32_t*>(&lo);
+      pk.y = *reinterpret_cast<uint32_t*>(&hi);
+      reinterpret_cast<uint2*>(a.shadow)[q * 32 + lane] = pk;
+    }
+  };
   int buf = 0;
-  if (PP > 0 && gw < nspan) issue(gw, stage);
+  if (gw < nspan) issue(gw, stage);
 
-  for (int64_t span = gw; span < nspan; span += nw, buf ^= (NBUF - 1)) {
+  for (int64_t span = gw; span < nspan; span += nw, buf ^= 1) {
     const int64_t q0 = span * S;
     const int nq = (int)min((int64_t)S, a.nblk - q0);
     float4* cur = stage + buf * S * 32;
+    if (span + nw < nspan) issue(span + nw, stage + (buf ^ 1) * S * 32);
+    else asm volatile("cp.async.commit_group;" ::: "memory");
     // segment of the span's first block; segments start on block boundaries
-    int seg = 0;
-    while (seg + 1 < a.nseg && q0 * 128 >= a.seg_off[seg + 1]) ++seg;
-    const int pmax = PP > 0 ? PP : a.pmax;
-    for (int p0 = 0; p0 < a.n; p0 += pmax) {
-      const int np = min(pmax, a.n - p0);
-      const bool last_pass = p0 + pmax >= a.n;
-      if (PP == 0) {
-        // theta loads land during the sign phase (a later pass re-reads what
-        // this lane stored in the previous one)
-        if (p0 > 0) __threadfence_block();
-        issue(span, cur);
-      }
-      const int pairs = np * S;
-#pragma unroll 4
-      for (int t = lane; t < pairs; t += 32) {
-        const int i = t / S, b = t - i * S;
-        if (b < nq) words[t] = sign_block(a.seed, (uint32_t)(p0 + i), (uint64_t)(q0 + b));
-      }
-      if (PP > 0) {
-        // next span's theta into the other buffer, then wait for this span's
-        if (span + nw < nspan) issue(span + nw, stage + (buf ^ 1) * S * 32);
-        else asm volatile("cp.async.commit_group;" ::: "memory");
-        asm volatile("cp.async.wait_group 1;" ::: "memory");
-      } else {
-        asm volatile("cp.async.wait_all;" ::: "memory");
-      }
-      __syncwarp();
-      int sg = seg;
-      for (int it = 0; it < nq; ++it) {
-        const int64_t q = q0 + it;
-        const float4 th = cur[it * 32 + lane];
-        double acc0 = th.x, acc1 = th.y, acc2 = th.z, acc3 = th.w;
-        const uint32_t* wcol = words32 + it * 4 + widx;
-        if constexpr (PP > 0) {
+    int sg = 0;
+    while (sg + 1 < a.nseg && q0 * 128 >= a.seg_off[sg + 1]) ++sg;
+    double acc[MULTI ? S : 1][4];
+    for (int ch = 0; ch < (MULTI ? a.chunks : 1); ++ch) {
+      // sign phase
+      if (lane < PAIRS && pb < nq) {
+        const int pbase = (ch * NG + pg) * 4;
+        // all four blocks unconditionally (independent chains interleave);
+        // probes past n_pert are zeroed afterwards
+        uint4 w[4];
 #pragma unroll
-          for (int g = 0; g < PP; g += 8) {
-            float2 s01 = make_float2(0.f, 0.f), s23 = make_float2(0.f, 0.f);
+        for (int r = 0; r < 4; ++r) w[r] = sign_block(a.seed, (uint32_t)(pbase + r), (uint64_t)(q0 + pb));
 #pragma unroll
-            for (int i = g; i < g + 8; ++i) {
-              const uint32_t w = wcol[i * SC * 4] >> sh;
-              s01 = add_f32x2(s01, make_float2(flip_sign(ncr[i], w << 31), flip_sign(ncr[i], w << 15)));
-              s23 = add_f32x2(s23, make_float2(flip_sign(ncr[i], w << 30), flip_sign(ncr[i], w << 14)));
-            }
-            acc0 += s01.x;
-            acc1 += s01.y;
-            acc2 += s23.x;
-            acc3 += s23.y;
-          }
-        } else {
-          for (int g = 0; g < np; g += 8) {
-            float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-            const int ge = min(g + 8, np);
-#pragma unroll 8
-            for (int i = g; i < ge; ++i) {
-              const float nc = negc[p0 + i];
-              const uint32_t w = wcol[i * S * 4] >> sh;
-              s0 += flip_sign(nc, w << 31);
-              s1 += flip_sign(nc, w << 15);
-              s2 += flip_sign(nc, w << 30);
-              s3 += flip_sign(nc, w << 14);
-            }
-            acc0 += s0;
-            acc1 += s1;
-            acc2 += s2;
-            acc3 += s3;
-          }
-        }
-        while (sg + 1 < a.nseg && q * 128 >= a.seg_off[sg + 1]) ++sg;
-        const int64_t j = q * 128 + 4 * lane;
-        const int64_t lim = a.seg_end[sg];
-        float4 o;
-        o.x = j + 0 < lim ? (float)acc0 : th.x;
-        o.y = j + 1 < lim ? (float)acc1 : th.y;
-        o.z = j + 2 < lim ? (float)acc2 : th.z;
-        o.w = j + 3 < lim ? (float)acc3 : th.w;
-        reinterpret_cast<float4*>(a.theta)[q * 32 + lane] = o;
-        if (last_pass && a.shadow) {
-          __nv_bfloat162 lo = __floats2bfloat162_rn(o.x, o.y);
-          __nv_bfloat162 hi = __floats2bfloat162_rn(o.z, o.w);
-          uint2 pk;
-          pk.x = *reinterpret_cast<uint32_t*>(&lo);
-          pk.y = *reinterpret_cast<uint32_t*>(&hi);
-          reinterpret_cast<uint2*>(a.shadow)[q * 32 + lane] = pk;
+        for (int r = 0; r < 4; ++r)
+          if (pbase + r >= a.n) w[r] = make_uint4(0u, 0u, 0u, 0u);
+        uint2* dst = idxw + lane * kPairStride;
+#pragma unroll
+        for (int wi = 0; wi < 4; ++wi) {
+          uint32_t W[8];
+          index_bytes(word_of(w[0], wi), word_of(w[1], wi), word_of(w[2], wi), word_of(w[3], wi), W);
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc) dst[wi * 4 + cc] = make_uint2(W[2 * cc], W[2 * cc + 1]);
         }
       }
+      if (ch == 0) asm volatile("cp.async.wait_group 1;" ::: "memory");
       __syncwarp();
+      // apply phase
+      const float* tabc = tab + ch * NG * 16;
+#pragma unroll
+      for (int it = 0; it < S; ++it) {
+        if (it < nq) {
+          float2 v01[NG], v23[NG];
+#pragma unroll
+          for (int g = 0; g < NG; ++g) {
+            const uint2 wv = idxw[(g * S + it) * kPairStride + unit];
+            const float* tg = tabc + g * 16;
+            v01[g] = make_float2(table_at(tg, __byte_perm(wv.x, 0u, sel_lo)),
+                                 table_at(tg, __byte_perm(wv.x, 0u, sel_hi)));
+            v23[g] = make_float2(table_at(tg, __byte_perm(wv.y, 0u, sel_lo)),
+                                 table_at(tg, __byte_perm(wv.y, 0u, sel_hi)));
+          }
+#pragma unroll
+          for (int w = 1; w < NG; w *= 2) {
+#pragma unroll
+            for (int g = 0; g + w < NG; g += 2 * w) {
+              v01[g] = add_f32x2(v01[g], v01[g + w]);
+              v23[g] = add_f32x2(v23[g], v23[g + w]);
+            }
+          }
+          const float4 th = cur[it * 32 + lane];
+          if constexpr (MULTI) {
+            if (ch == 0) {
+              acc[it][0] = th.x;
+              acc[it][1] = th.y;
+              acc[it][2] = th.z;
+              acc[it][3] = th.w;
+            }
+            acc[it][0] += v01[0].x;
+            acc[it][1] += v01[0].y;
+            acc[it][2] += v23[0].x;
+            acc[it][3] += v23[0].y;
+          } else {
+            const float2 o01 = add_f32x2(make_float2(th.x, th.y), v01[0]);
+            const float2 o23 = add_f32x2(make_float2(th.z, th.w), v23[0]);
+            write_out(q0 + it, sg, th, make_float4(o01.x, o01.y, o23.x, o23.y));
+          }
+        }
+      }
+      __syncwarp();   // the next pass's sign phase reuses the index words
     }
+    if constexpr (MULTI) {
+#pragma unroll
+      for (int it = 0; it < S; ++it) {
+        if (it < nq)
+          write_out(q0 + it, sg, cur[it * 32 + lane],
+                    make_float4((float)acc[it][0], (float)acc[it][1], (float)acc[it][2],
+                                (float)acc[it][3]));
+      }
+    }
+    __syncwarp();
   }
 }
 
-template <int PP>
-static cudaError_t launch_update_pp(const UpdateArgs& a, int sm_count, cudaStream_t st) {
-  const int ncap = PP > 0 ? PP : a.n;
-  const size_t wslots = PP > 0 ? (size_t)PP * a.S : (size_t)kUpdSlots;
-  const size_t smem = sizeof(uint4) * ((ncap + 3) / 4 + (size_t)kUpdWarps * wslots +
-                                      (size_t)kUpdWarps * (PP > 0 ? 2 : 1) * a.S * 32);
-  cudaFuncSetAttribute(update_kernel<PP>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  cudaFuncSetAttribute(update_kernel<PP>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-  const int64_t nspan = (a.nblk + a.S - 1) / a.S;
+template <int NG, bool MULTI>
+static cudaError_t launch_update_ng(const UpdateArgs& a, int sm_count, cudaStream_t st) {
+  constexpr int S = NG >= 4 ? 32 / NG : 8;
+  const size_t smem = (size_t)a.ngroups * 64 + (size_t)kUpdWarps * 32 * kPairStride * 8 +
+                      (size_t)kUpdWarps * 2 * S * 32 * 16;
+  cudaFuncSetAttribute(update_kernel<NG, MULTI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       (int)smem);
+  cudaFuncSetAttribute(update_kernel<NG, MULTI>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                       100);
+  const int64_t nspan = (a.nblk + S - 1) / S;
   int64_t grid = (nspan + kUpdWarps - 1) / kUpdWarps;
-  int per_sm = (int)((220 * 1024) / smem);
-  if (per_sm < 1) per_sm = 1;
-  if (per_sm > 8) per_sm = 8;
+  // one resident wave: blocks per SM as registers and shared memory allow
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, update_kernel<NG, MULTI>,
+                                                    kUpdWarps * 32, smem) != cudaSuccess ||
+      per_sm < 1)
+    per_sm = 1;
   const int64_t cap = (int64_t)sm_count * per_sm;
   if (grid > cap) grid = cap;
-  update_kernel<PP><<<(int)grid, kUpdWarps * 32, smem, st>>>(a);
+  update_kernel<NG, MULTI><<<(int)grid, kUpdWarps * 32, smem, st>>>(a);
   count_launch();
   return cudaGetLastError();
 }
@@ -315,27 +372,22 @@ cudaError_t launch_update(const zo_ctx* ctx, float* theta, uint64_t seed, int n,
     a.seg_end[s] = ctx->seg.off[s] + ctx->seg.numel[s];
   }
   a.err = ctx->err;
-  const int64_t want = (int64_t)ctx->sm_count * 16;   // spans that fill the GPU
-  // compile-time probe counts for large models
-  const int pp = n <= 16 ? 16 : n <= 32 ? 32 : n <= 64 ? 64 : 0;
-  if (pp) {
-    const int S = 128 / pp < 32 ? 128 / pp : 32;
-    if ((a.nblk + S - 1) / S >= want) {
-      a.S = S;
-      a.pmax = pp;
-      if (pp == 16) return launch_update_pp<16>(a, ctx->sm_count, st);
-      if (pp == 32) return launch_update_pp<32>(a, ctx->sm_count, st);
-      return launch_update_pp<64>(a, ctx->sm_count, st);
+  const int ng = (n + 3) / 4;
+  if (ng <= 16) {
+    const int NG = ng <= 1 ? 1 : ng <= 2 ? 2 : ng <= 4 ? 4 : ng <= 8 ? 8 : 16;
+    a.ngroups = NG;
+    a.chunks = 1;
+    switch (NG) {
+      case 1: return launch_update_ng<1, false>(a, ctx->sm_count, st);
+      case 2: return launch_update_ng<2, false>(a, ctx->sm_count, st);
+      case 4: return launch_update_ng<4, false>(a, ctx->sm_count, st);
+      case 8: return launch_update_ng<8, false>(a, ctx->sm_count, st);
+      default: return launch_update_ng<16, false>(a, ctx->sm_count, st);
     }
   }
-  // blocks per span: all probes in one pass if possible, and enough spans
-  // to give every SM 16 warps of work
-  int S = 32;
-  while (S > 1 && S * n > kUpdSlots) S /= 2;
-  while (S > 1 && (a.nblk + S - 1) / S < want) S /= 2;
-  a.S = S;
-  a.pmax = kUpdSlots / S < n ? kUpdSlots / S : n;
-  return launch_update_pp<0>(a, ctx->sm_count, st);
+  a.chunks = (ng + 15) / 16;
+  a.ngroups = a.chunks * 16;
+  return launch_update_ng<16, true>(a, ctx->sm_count, st);
 }
 
 }  // namespace zo

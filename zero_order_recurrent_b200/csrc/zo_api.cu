@@ -371,7 +371,7 @@ int zo_coeffs(zo_ctx* ctx, const float* lp, const float* lm, int32_t n, float ep
 
 int zo_update(zo_ctx* ctx, float* theta, uint64_t seed, int32_t n, const float* coeffs,
               void* stream) {
-  if (!ctx || !theta || !coeffs || n < 1) return ZO_ERR_INVALID_ARG;
+  if (!ctx || !theta || !coeffs || n < 1 || n > ZO_MAX_UPDATE_PROBES) return ZO_ERR_INVALID_ARG;
   __nv_bfloat16* sh = ctx->spec.dtype == ZO_DTYPE_BF16 ? ctx->shadow : nullptr;
   const double bytes = (double)ctx->seg.d_pad * (sh ? 10.0 : 8.0);
   ZO_CUDA(timed(ctx, S(stream), ZO_KIND_UPDATE, 0.0, bytes,
