@@ -198,6 +198,11 @@ def test_fp32_overfit_full_launch_sampled_probes():
     (13, 8, 24, 2, 9, 3, 7, 3, 0.5),    # ragged row blocks, several chunks
     (11, 12, 40, 1, 1, 1, 1, 0, 0.0),   # T = 1, one probe
     (9, 4, 8, 2, 3, 5, 2, 0, 1.0),      # nothing scored: loss 0
+    # widths that are multiples of 32 take the probe-column kernel (four
+    # probes per CTA, rows across lanes):
+    (50, 32, 32, 1, 3, 4, 6, 0, 0.3),   # inputs split over warps, a CTA with 2 of 4 probes
+    (65, 64, 64, 2, 2, 3, 5, 2, 0.0),   # 65 logits (two row blocks), split inputs, chunks
+    (40, 96, 96, 3, 1, 5, 9, 0, 0.5),   # three layers, 6 row blocks, 3 input words
 ])
 def test_fp32_edge_cases(V, E, H, L, B, T, n, chunk, frac):
     cfg = W.small_config(vocab=V, embed=E, hidden=H, layers=L)

@@ -16,7 +16,6 @@
 
 namespace zo {
 std::atomic<int64_t> g_launches{0};
-size_t fp32_smem_bytes(const zo_model_spec& s, int bb, int64_t d_pad);
 }  // namespace zo
 
 using namespace zo;
@@ -101,6 +100,7 @@ void free_ctx(zo_ctx* c) {
   cudaFree(c->lp);
   cudaFree(c->lm);
   cudaFree(c->coef);
+  cudaFree(c->wt);
   for (auto& r : c->prof) {
     if (r.a) cudaEventDestroy(r.a);
     if (r.b) cudaEventDestroy(r.b);
@@ -184,13 +184,22 @@ int zo_create(const zo_model_spec* spec, zo_ctx** out) {
     // (the probe's sign words for all d_pad parameters live in shared memory)
     const int64_t dp = c->seg.d_pad;
     int bb = 8;
-    while (bb > 1 && (bb / 2 >= B || fp32_smem_bytes(s, bb, dp) > 200 * 1024)) bb /= 2;
-    if (fp32_smem_bytes(s, bb, dp) > 200 * 1024) {
+    while (bb > 1 && (bb / 2 >= B || fp32_smem_bytes(s, bb, 1, dp) > 200 * 1024)) bb /= 2;
+    if (fp32_smem_bytes(s, bb, 1, dp) > 200 * 1024) {
       free_ctx(c);
       return ZO_ERR_UNSUPPORTED;
     }
     c->fp32_bb = bb;
-    c->fp32_smem = fp32_smem_bytes(s, bb, dp);
+    c->fp32_smem = fp32_smem_bytes(s, bb, 1, dp);
+    // probe-column forward (several probes share each weight load) where the
+    // shape and shared memory allow; it needs a transposed copy of W
+    int64_t wt_floats = 0;
+    size_t wide_smem = 0;
+    const int wnp = fp32_wide_probes(s, 220 * 1024, &wt_floats, &wide_smem);
+    if (wnp > 0) {
+      alloc((void**)&c->wt, sizeof(float) * (size_t)wt_floats);
+      c->fp32_wide_np = wnp;
+    }
     c->chunk = s.chunk > 0 ? s.chunk : 4096;
     alloc((void**)&c->rowloss, sizeof(float) * 2 * (size_t)c->chunk * B);
   } else {
@@ -294,8 +303,11 @@ static int probe_losses_range(zo_ctx* ctx, const float* theta, uint64_t seed, in
       const int np = n_pert - p0 < ctx->chunk ? n_pert - p0 : ctx->chunk;
       const double fl = 2.0 * 2 * np * (double)B * T * fwd_macs;
       ZO_CUDA(timed(ctx, st, ZO_KIND_CELL, fl, 0.0, [&] {
-        return launch_fp32_forward(ctx, theta, seed, probe_begin + p0, np, eps, tokens, targets, B,
-                                   T, st);
+        return ctx->fp32_wide_np
+                   ? launch_fp32_wide(ctx, theta, seed, probe_begin + p0, np, eps, tokens, targets,
+                                      B, T, st)
+                   : launch_fp32_forward(ctx, theta, seed, probe_begin + p0, np, eps, tokens,
+                                         targets, B, T, st);
       }));
       ZO_CUDA(timed(ctx, st, ZO_KIND_OTHER, 0.0, 0.0, [&] {
         return launch_reduce_losses(ctx, targets, B, T, p0, np, loss_plus, loss_minus, row_loss, st);

@@ -77,6 +77,8 @@ struct zo_ctx {
   int n_stage = 0;               // capacity of lp/lm/coef
   int fp32_bb = 1;               // rows per CTA of the fp32 forward
   size_t fp32_smem = 0;
+  int fp32_wide_np = 0;          // probes per CTA of the probe-column fp32 forward (0: unused)
+  float* wt = nullptr;           // its transposed weight copies
   // per-launch timing (zo_profile)
   bool prof_on = false;
   std::vector<ZoProfRec> prof;
@@ -114,6 +116,13 @@ cudaError_t launch_cell_tc(const zo_ctx* ctx, int layer, int t, int B, int nprob
                            uint64_t seed, float eps, float* raw_out, cudaStream_t st);
 bool make_cell_maps(zo_ctx* ctx);
 void layout_of(const zo_model_spec& sp, Segments& s);
-size_t fp32_smem_bytes(const zo_model_spec& s, int bb, int64_t d_pad);
+// probe-column fp32 forward: probes per CTA that fit `limit` bytes of shared
+// memory (0 if the shape is not supported), its workspace and shared memory
+int fp32_wide_probes(const zo_model_spec& s, size_t limit, int64_t* wt_floats, size_t* smem);
+cudaError_t launch_fp32_wide(const zo_ctx* ctx, const float* theta, uint64_t seed, int probe0,
+                             int nprobe, float eps, const int32_t* tokens, const int32_t* targets,
+                             int B, int T, cudaStream_t st);
+// shared memory of the fp32 forward for bb batch rows x np probes per CTA
+size_t fp32_smem_bytes(const zo_model_spec& s, int bb, int np, int64_t d_pad);
 
 }  // namespace zo
