@@ -276,7 +276,11 @@ def roofline_for(cfg, kinds, clocks, pk):
     achieved = fl_cell / (ms_cell / 1e3) / 1e12
     mhz = pk["sm_max_mhz"]
     peak = fp32_alu_peak_tflops(mhz)
-    return {"bound": "alu", "kernel": "fp32_forward_kernel (persistent perturbed LSTM forward)",
+    # the context takes the probe-column kernel when E and H are multiples of 32
+    wide = cfg.embed % 32 == 0 and cfg.hidden % 32 == 0
+    name = ("fp32_wide_kernel (probe-column perturbed LSTM forward, 4 probes per CTA)" if wide
+            else "fp32_forward_kernel (persistent perturbed LSTM forward)")
+    return {"bound": "alu", "kernel": name,
             "achieved": round(achieved, 3), "peak": round(peak, 2), "unit": "TFLOP/s",
             "frac": round(achieved / peak, 4), "traffic": captured_traffic(cfg),
             "peak_source": f"fp32 FMA: 148 SMs x 128 lanes x 2 x {mhz:.0f} MHz",
