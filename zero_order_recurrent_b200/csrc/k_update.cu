@@ -220,15 +220,19 @@ __global__ void __launch_bounds__(kUpdWarps * 32, 4) update_kernel(const UpdateA
   };
   // theta' of block q: pads past the block's segment end keep theta, and the
   // bf16 shadow gets the same values
-  auto write_out = [&](int64_t q, int& sg, float4 th, float4 o) {
-    while (sg + 1 < a.nseg && q * 128 >= a.seg_off[sg + 1]) ++sg;
-    const int64_t lim = a.seg_end[sg];
-    if (q * 128 + 128 > lim) {
-      const int64_t j = q * 128 + 4 * lane;
-      o.x = j + 0 < lim ? o.x : th.x;
-      o.y = j + 1 < lim ? o.y : th.y;
-      o.z = j + 2 < lim ? o.z : th.z;
-      o.w = j + 3 < lim ? o.w : th.w;
+  // (clean: the whole span lies inside one segment's real entries, so no
+  // block needs the search or the mask)
+  auto write_out = [&](int64_t q, int& sg, bool clean, float4 th, float4 o) {
+    if (!clean) {
+      while (sg + 1 < a.nseg && q * 128 >= a.seg_off[sg + 1]) ++sg;
+      const int64_t lim = a.seg_end[sg];
+      if (q * 128 + 128 > lim) {
+        const int64_t j = q * 128 + 4 * lane;
+        o.x = j + 0 < lim ? o.x : th.x;
+        o.y = j + 1 < lim ? o.y : th.y;
+        o.z = j + 2 < lim ? o.z : th.z;
+        o.w = j + 3 < lim ? o.w : th.w;
+      }
     }
     reinterpret_cast<float4*>(a.theta)[q * 32 + lane] = o;
     if (a.shadow) {
@@ -252,6 +256,7 @@ __global__ void __launch_bounds__(kUpdWarps * 32, 4) update_kernel(const UpdateA
     // segment of the span's first block; segments start on block boundaries
     int sg = 0;
     while (sg + 1 < a.nseg && q0 * 128 >= a.seg_off[sg + 1]) ++sg;
+    const bool clean = (q0 + nq) * 128 <= a.seg_end[sg];
     double acc[MULTI ? S : 1][4];
     for (int ch = 0; ch < (MULTI ? a.chunks : 1); ++ch) {
       // sign phase
@@ -314,7 +319,7 @@ __global__ void __launch_bounds__(kUpdWarps * 32, 4) update_kernel(const UpdateA
           } else {
             const float2 o01 = add_f32x2(make_float2(th.x, th.y), v01[0]);
             const float2 o23 = add_f32x2(make_float2(th.z, th.w), v23[0]);
-            write_out(q0 + it, sg, th, make_float4(o01.x, o01.y, o23.x, o23.y));
+            write_out(q0 + it, sg, clean, th, make_float4(o01.x, o01.y, o23.x, o23.y));
           }
         }
       }
@@ -324,7 +329,7 @@ __global__ void __launch_bounds__(kUpdWarps * 32, 4) update_kernel(const UpdateA
 #pragma unroll
       for (int it = 0; it < S; ++it) {
         if (it < nq)
-          write_out(q0 + it, sg, cur[it * 32 + lane],
+          write_out(q0 + it, sg, clean, cur[it * 32 + lane],
                     make_float4((float)acc[it][0], (float)acc[it][1], (float)acc[it][2],
                                 (float)acc[it][3]));
       }
