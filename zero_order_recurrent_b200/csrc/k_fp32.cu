@@ -1,18 +1,17 @@
 // fp32 CUDA-core path for small models: one persistent CTA runs the whole
-// sequence for NP probes (both signs each) and a slice of BB batch rows, with
-// the recurrent state in shared memory and the perturbed weights W +- eps P
+// sequence for one probe (both signs) and a slice of the batch, with the
+// recurrent state in shared memory and the perturbed weights W +- eps P
 // formed on the fly.  Every cell step is
 //   G = [x_t | h_{t-1}] (W +- eps P)^T + (b +- eps p),
 //   c_t = sigma(f) c_{t-1} + sigma(i) tanh(g),  h_t = sigma(o) tanh(c_t)
 // (pith.science review, "What carries the argument": complete forwards at
 // Theta +- eps p_i; cell and loss readings in the oracle's header).
 //
-// The sign words of the CTA's probes for the whole parameter vector (d/8
-// bytes per probe) are generated once into shared memory, so the timestep
-// loop runs no Philox at all.  Weight rows are read by groups of 8 lanes
-// (float4 each, 128 contiguous bytes per row), so every global load is
-// coalesced; each weight load serves all NP x BB (probe, row) pairs of the
-// CTA and both signs, which divides the weight traffic from L2 by NP x BB.
+// The probe's sign words for the whole parameter vector (d/8 bytes) are
+// generated once per CTA into shared memory, so the timestep loop runs no
+// Philox at all.  Weight rows are read by groups of 8 lanes (float4 each,
+// 128 contiguous bytes per row), so every global load is coalesced; the two
+// signs share each weight load and each sign word.
 #include "zo_common.cuh"
 #include "zo_internal.h"
 
@@ -25,7 +24,6 @@ struct Fp32Args {
   float eps;
   const int32_t* tokens;
   const int32_t* targets;
-  int nprobe;      // probes of this launch (CTAs past it mask their tail)
   int B, T, Bmax;
   int V, E, H, L;
   int64_t nblk;    // d_pad / 128
@@ -35,15 +33,6 @@ struct Fp32Args {
 };
 
 constexpr int kFpThreads = 256;
-#ifndef ZO_FP32_MAX_PROBES
-#define ZO_FP32_MAX_PROBES 1
-#endif
-constexpr int kFp32MaxProbes = ZO_FP32_MAX_PROBES;   // probes per CTA (power of two)
-constexpr size_t kFp32SmemLimit = 220 * 1024;
-#ifndef ZO_FP32_MIN_CTAS
-#define ZO_FP32_MIN_CTAS 0
-#endif
-constexpr int kFp32MinCtasPerSm = ZO_FP32_MIN_CTAS;
 
 // Signed perturbation +-eps for element j from the shared sign words.
 __device__ __forceinline__ float pert(const uint32_t* sw, int64_t j, float eps) {
@@ -70,8 +59,7 @@ __device__ __forceinline__ float2 add_f32x2(float2 a, float2 b) {
 }
 
 // Subset-sum tables for the probe term.  For the concatenated input
-// a = [in | rec] of one step, every (probe, row) pair b of the CTA and every
-// group g of 4 inputs (k = 4g..4g+3),
+// a = [in | rec] of one step and every group g of 4 inputs (k = 4g..4g+3),
 //   U[b][g][idx] = ( sum_k p_k a+_k,  -sum_k p_k a-_k )  over the group,
 // where p_k = -1 for the elements whose bit is set in the 4-bit index idx
 // (bit 0 <-> k = 4g, bit 1 <-> 4g+2, bit 2 <-> 4g+1, bit 3 <-> 4g+3: the order
@@ -79,10 +67,10 @@ __device__ __forceinline__ float2 add_f32x2(float2 a, float2 b) {
 // Then sum_k p_k a_k over a row is one table lookup per group.
 constexpr int kUStride = 17;  // float2 per group (16 + 1 pad against bank conflicts)
 
-template <int NQ>
+template <int BB>
 __device__ void build_tables(const float* in, int Kin, const float* rec, int Krec, float2* U) {
   const int G = (Kin + Krec) / 4;
-  for (int e = threadIdx.x; e < NQ * G * 16; e += blockDim.x) {
+  for (int e = threadIdx.x; e < BB * G * 16; e += blockDim.x) {
     const int idx = e & 15;
     const int g = (e >> 4) % G;
     const int b = (e >> 4) / G;
@@ -90,10 +78,10 @@ __device__ void build_tables(const float* in, int Kin, const float* rec, int Kre
     float4 xp, xm;
     if (k < Kin) {
       xp = *reinterpret_cast<const float4*>(in + b * Kin + k);
-      xm = *reinterpret_cast<const float4*>(in + (NQ + b) * Kin + k);
+      xm = *reinterpret_cast<const float4*>(in + (BB + b) * Kin + k);
     } else {
       xp = *reinterpret_cast<const float4*>(rec + b * Krec + k - Kin);
-      xm = *reinterpret_cast<const float4*>(rec + (NQ + b) * Krec + k - Kin);
+      xm = *reinterpret_cast<const float4*>(rec + (BB + b) * Krec + k - Kin);
     }
     const float s0 = (idx & 1) ? -1.f : 1.f, s2 = (idx & 2) ? -1.f : 1.f;
     const float s1 = (idx & 4) ? -1.f : 1.f, s3 = (idx & 8) ? -1.f : 1.f;
@@ -103,27 +91,24 @@ __device__ void build_tables(const float* in, int Kin, const float* rec, int Kre
   }
 }
 
-// Rows [0, R) of a perturbed matrix-vector product for the NQ = NP x BB
-// (probe, row) pairs of the CTA and both signs.  Row r of the matrix starts at
-// theta[j0 + r*K]; its first Kin entries multiply `in` ([2][NQ][Kin] in shared
-// memory) and the rest `rec` ([2][NQ][K-Kin]).  Pair q = p*BB + b uses the
-// sign words of probe p (sw + p*sw_stride).
-//   out[s][q][r] = bias_s[r] + sum_k (W +- eps P_p)[r,k] a_s[q,k].
+// Rows [0, R) of a perturbed matrix-vector product for BB batch rows and both
+// signs.  Row r of the matrix starts at theta[j0 + r*K]; its first Kin entries
+// multiply `in` ([2][BB][Kin] in shared memory) and the rest `rec`
+// ([2][BB][K-Kin]).  out[s][b][r] = bias_s[r] + sum_k (W +- eps P)[r,k] a_s[b,k].
 //
 // VEC (rows and both parts 4-aligned): a lane is (k-slice l8 = lane & 7,
-// row slot rs = lane >> 3) and owns rows rb + rs + 4m, m < RPL (2 when NQ = 1,
-// else 1); it walks the groups g = l8 + 8i of 4 inputs, loads the group's
-// weights once and uses them for every pair: W a+- with packed fp32x2 FMAs on
-// (even, odd) pairs, eps P a+- from the subset-sum tables U.  Weight loads stay
-// coalesced (8 lanes x 16 B of one row).
-// Otherwise (NP = 1 only): 8 lanes per row, one element per step, W +- eps p
-// formed directly.
-template <int NP, int BB, bool VEC>
-__device__ void perturbed_gemv(const Fp32Args& a, const uint32_t* sw, int sw_stride, int64_t j0,
-                               int R, int K, int Kin, const float* in, const float* rec,
-                               const float2* U, int64_t jbias, float* out, int out_stride) {
-  constexpr int NQ = NP * BB;
-  constexpr int RPL = (VEC && NQ == 1) ? 2 : 1;   // rows per lane
+// row slot rs = lane >> 3) and owns rows rb + rs + 4m, m < RPL (2 when BB = 1,
+// else 1); it walks the
+// groups g = l8 + 8i of 4 inputs, loads the group's activations once and uses
+// them for all its rows: W a+- with packed fp32x2 FMAs on (even, odd) pairs,
+// eps P a+- from the subset-sum tables U.  Weight loads stay coalesced (8
+// lanes x 16 B of one row).
+// Otherwise: 8 lanes per row, one element per step, W +- eps p formed directly.
+template <int BB, bool VEC>
+__device__ void perturbed_gemv(const Fp32Args& a, const uint32_t* sw, int64_t j0, int R, int K,
+                               int Kin, const float* in, const float* rec, const float2* U,
+                               int64_t jbias, float* out, int out_stride) {
+  constexpr int RPL = (VEC && BB == 1) ? 2 : 1;   // rows per lane
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int nw = blockDim.x >> 5;
@@ -131,10 +116,10 @@ __device__ void perturbed_gemv(const Fp32Args& a, const uint32_t* sw, int sw_str
   const int Krec = K - Kin;
   const float eps = a.eps;
   for (int rb = warp * 4 * RPL; rb < R; rb += nw * 4 * RPL) {
-    float gp[RPL][NQ], gm[RPL][NQ];
+    float gp[RPL][BB], gm[RPL][BB];
     if (VEC) {
       const int G = K / 4, Gin = Kin / 4;
-      float2 wp[RPL][NQ], wm[RPL][NQ], pe[RPL][NQ];
+      float2 wp[RPL][BB], wm[RPL][BB], pe[RPL][BB];
       // row m of this lane: weights at wbase + roff[m] (float4 units), sign
       // word index wi[m] (+1 per step of 32 inputs), in-word shift sh[m]
       const float4* wbase = reinterpret_cast<const float4*>(a.theta + j0 + 4 * l8);
@@ -148,51 +133,48 @@ __device__ void perturbed_gemv(const Fp32Args& a, const uint32_t* sw, int sw_str
         wi[m] = (int)(jl >> 5);
         sh[m] = (int)(jl & 31) >> 1;
 #pragma unroll
-        for (int q = 0; q < NQ; ++q) wp[m][q] = wm[m][q] = pe[m][q] = make_float2(0.f, 0.f);
+        for (int b = 0; b < BB; ++b) wp[m][b] = wm[m][b] = pe[m][b] = make_float2(0.f, 0.f);
       }
       for (int g = l8; g < G; g += 8) {
-        float4 xp[NQ], xm[NQ];
+        float4 xp[BB], xm[BB];
 #pragma unroll
-        for (int q = 0; q < NQ; ++q) {
-          const float* src = g < Gin ? in + q * Kin + 4 * g : rec + q * Krec + 4 * g - Kin;
-          const int off = g < Gin ? NQ * Kin : NQ * Krec;
-          xp[q] = *reinterpret_cast<const float4*>(src);
-          xm[q] = *reinterpret_cast<const float4*>(src + off);
+        for (int b = 0; b < BB; ++b) {
+          const float* src = g < Gin ? in + b * Kin + 4 * g : rec + b * Krec + 4 * g - Kin;
+          const int off = g < Gin ? BB * Kin : BB * Krec;
+          xp[b] = *reinterpret_cast<const float4*>(src);
+          xm[b] = *reinterpret_cast<const float4*>(src + off);
         }
 #pragma unroll
         for (int m = 0; m < RPL; ++m) {
           const float4 w = __ldg(wbase + roff[m] + (g - l8));
-          int idx[NP];
+          const uint32_t s = sw[wi[m] + ((g - l8) >> 3)] >> sh[m];
+          const int idx = (int)((s & 3u) | ((s >> 14) & 12u));
 #pragma unroll
-          for (int p = 0; p < NP; ++p) {
-            const uint32_t s = sw[p * sw_stride + wi[m] + ((g - l8) >> 3)] >> sh[m];
-            idx[p] = (int)((s & 3u) | ((s >> 14) & 12u));
-          }
-#pragma unroll
-          for (int q = 0; q < NQ; ++q) {
-            wp[m][q] = fma_f32x2(make_float2(w.x, w.y), make_float2(xp[q].x, xp[q].y), wp[m][q]);
-            wp[m][q] = fma_f32x2(make_float2(w.z, w.w), make_float2(xp[q].z, xp[q].w), wp[m][q]);
-            wm[m][q] = fma_f32x2(make_float2(w.x, w.y), make_float2(xm[q].x, xm[q].y), wm[m][q]);
-            wm[m][q] = fma_f32x2(make_float2(w.z, w.w), make_float2(xm[q].z, xm[q].w), wm[m][q]);
-            pe[m][q] = add_f32x2(pe[m][q], U[(q * G + g) * kUStride + idx[q / BB]]);
+          for (int b = 0; b < BB; ++b) {
+            wp[m][b] = fma_f32x2(make_float2(w.x, w.y), make_float2(xp[b].x, xp[b].y), wp[m][b]);
+            wp[m][b] = fma_f32x2(make_float2(w.z, w.w), make_float2(xp[b].z, xp[b].w), wp[m][b]);
+            wm[m][b] = fma_f32x2(make_float2(w.x, w.y), make_float2(xm[b].x, xm[b].y), wm[m][b]);
+            wm[m][b] = fma_f32x2(make_float2(w.z, w.w), make_float2(xm[b].z, xm[b].w), wm[m][b]);
+            pe[m][b] = add_f32x2(pe[m][b], U[(b * G + g) * kUStride + idx]);
           }
         }
       }
 #pragma unroll
       for (int m = 0; m < RPL; ++m)
 #pragma unroll
-        for (int q = 0; q < NQ; ++q) {
-          gp[m][q] = fmaf(eps, pe[m][q].x, wp[m][q].x + wp[m][q].y);
-          gm[m][q] = fmaf(eps, pe[m][q].y, wm[m][q].x + wm[m][q].y);
+        for (int b = 0; b < BB; ++b) {
+          gp[m][b] = fmaf(eps, pe[m][b].x, wp[m][b].x + wp[m][b].y);
+          gm[m][b] = fmaf(eps, pe[m][b].y, wm[m][b].x + wm[m][b].y);
         }
     } else {
       const int r = rb + (lane >> 3);
       const int64_t jr = j0 + (int64_t)(r < R ? r : 0) * K;
 #pragma unroll
-      for (int q = 0; q < NQ; ++q) gp[0][q] = gm[0][q] = 0.f;
+      for (int b = 0; b < BB; ++b) gp[0][b] = gm[0][b] = 0.f;
       if (r < R) {
         for (int k = l8; k < K; k += 8) {
           const float w = __ldg(a.theta + jr + k);
+          const float d = pert(sw, jr + k, eps);
           const float* src;
           int ld, kk;
           if (k < Kin) {
@@ -205,10 +187,9 @@ __device__ void perturbed_gemv(const Fp32Args& a, const uint32_t* sw, int sw_str
             kk = k - Kin;
           }
 #pragma unroll
-          for (int q = 0; q < NQ; ++q) {
-            const float d = pert(sw + (q / BB) * sw_stride, jr + k, eps);
-            gp[0][q] = fmaf(w + d, src[q * ld + kk], gp[0][q]);
-            gm[0][q] = fmaf(w - d, src[(NQ + q) * ld + kk], gm[0][q]);
+          for (int b = 0; b < BB; ++b) {
+            gp[0][b] = fmaf(w + d, src[b * ld + kk], gp[0][b]);
+            gm[0][b] = fmaf(w - d, src[(BB + b) * ld + kk], gm[0][b]);
           }
         }
       }
@@ -216,64 +197,54 @@ __device__ void perturbed_gemv(const Fp32Args& a, const uint32_t* sw, int sw_str
 #pragma unroll
     for (int m = 0; m < RPL; ++m) {
 #pragma unroll
-      for (int q = 0; q < NQ; ++q) {
+      for (int b = 0; b < BB; ++b) {
 #pragma unroll
         for (int o = 4; o > 0; o >>= 1) {
-          gp[m][q] += __shfl_xor_sync(0xffffffffu, gp[m][q], o);
-          gm[m][q] += __shfl_xor_sync(0xffffffffu, gm[m][q], o);
+          gp[m][b] += __shfl_xor_sync(0xffffffffu, gp[m][b], o);
+          gm[m][b] += __shfl_xor_sync(0xffffffffu, gm[m][b], o);
         }
       }
       const int r = rb + (lane >> 3) + 4 * m;
       if (r < R && l8 == 0) {
         const float bth = a.theta[jbias + r];
+        const float bd = pert(sw, jbias + r, eps);
 #pragma unroll
-        for (int q = 0; q < NQ; ++q) {
-          const float bd = pert(sw + (q / BB) * sw_stride, jbias + r, eps);
-          out[q * out_stride + r] = gp[m][q] + (bth + bd);
-          out[(NQ + q) * out_stride + r] = gm[m][q] + (bth - bd);
+        for (int b = 0; b < BB; ++b) {
+          out[b * out_stride + r] = gp[m][b] + (bth + bd);
+          out[(BB + b) * out_stride + r] = gm[m][b] + (bth - bd);
         }
       }
     }
   }
 }
 
-template <int NP, int BB, bool VEC>
-__global__ void __launch_bounds__(kFpThreads, NP * BB <= 2 ? 4 : 2)
-    fp32_forward_kernel(const Fp32Args a) {
-  constexpr int NQ = NP * BB;
+template <int BB, bool VEC>
+__global__ void __launch_bounds__(kFpThreads, BB <= 2 ? 4 : 2) fp32_forward_kernel(const Fp32Args a) {
   extern __shared__ __align__(16) float sm[];
-  const int pc = blockIdx.x * NP;              // first probe of this CTA (launch-local)
-  const int npv = min(NP, a.nprobe - pc);      // probes of the CTA inside the launch
+  const int ci = blockIdx.x;
+  const uint32_t probe = (uint32_t)(a.probe0 + ci);
   const int r0 = blockIdx.y * BB;
   const int nb = min(BB, a.B - r0);
   const int H = a.H, E = a.E, V = a.V, L = a.L;
   const int G4 = 4 * H;
   const int tid = threadIdx.x, nt = blockDim.x;
-  const int sw_stride = (int)(a.nblk * 4);
-  uint32_t* sw = reinterpret_cast<uint32_t*>(sm);          // [NP][nblk*4] sign words
-  float* xin = sm + NP * a.nblk * 4;                       // [2][NQ][E]
-  float* hs = xin + 2 * NQ * E;                            // [L][2][NQ][H]
-  float* cs = hs + L * 2 * NQ * H;                         // [L][2][NQ][H]
-  float* gs = cs + L * 2 * NQ * H;                         // [2][NQ][4H]
-  float* lg = gs + 2 * NQ * G4;                            // [2][NQ][V]
-  float* rl = lg + 2 * NQ * V;                             // [2][NQ]
-  float2* U = reinterpret_cast<float2*>(rl + ((2 * NQ + 3) & ~3));  // [NQ][Gmax][17] (VEC)
-  // probes past the launch (npv < NP) still run, on valid probe indices, and
-  // are never written out
-  for (int64_t e = tid; e < (int64_t)NP * a.nblk; e += nt) {
-    const int p = (int)(e / a.nblk);
-    const int64_t q = e - (int64_t)p * a.nblk;
-    const uint32_t probe = (uint32_t)(a.probe0 + pc + (p < npv ? p : 0));
-    reinterpret_cast<uint4*>(sw + p * sw_stride)[q] = sign_block(a.seed, probe, (uint64_t)q);
-  }
-  for (int i = tid; i < 2 * L * 2 * NQ * H; i += nt) hs[i] = 0.f;  // hs, cs
-  for (int i = tid; i < 2 * NQ; i += nt) rl[i] = 0.f;
+  uint32_t* sw = reinterpret_cast<uint32_t*>(sm);        // [nblk*4] sign words
+  float* xin = sm + a.nblk * 4;                            // [2][BB][E]
+  float* hs = xin + 2 * BB * E;                            // [L][2][BB][H]
+  float* cs = hs + L * 2 * BB * H;                         // [L][2][BB][H]
+  float* gs = cs + L * 2 * BB * H;                         // [2][BB][4H]
+  float* lg = gs + 2 * BB * G4;                            // [2][BB][V]
+  float* rl = lg + 2 * BB * V;                             // [2][BB]
+  float2* U = reinterpret_cast<float2*>(rl + ((2 * BB + 3) & ~3));  // [BB][Gmax][17] (VEC)
+  for (int64_t q = tid; q < a.nblk; q += nt)
+    reinterpret_cast<uint4*>(sw)[q] = sign_block(a.seed, probe, (uint64_t)q);
+  for (int i = tid; i < 2 * L * 2 * BB * H; i += nt) hs[i] = 0.f;  // hs, cs
+  for (int i = tid; i < 2 * BB; i += nt) rl[i] = 0.f;
   __syncthreads();
 
   for (int t = 0; t < a.T; ++t) {
-    for (int i = tid; i < NQ * E; i += nt) {
-      const int q = i / E, k = i % E;
-      const int b = q % BB;
+    for (int i = tid; i < BB * E; i += nt) {
+      const int b = i / E, k = i % E;
       float vp = 0.f, vm = 0.f;
       if (b < nb) {
         int tok = a.tokens[(int64_t)(r0 + b) * a.T + t];
@@ -282,50 +253,48 @@ __global__ void __launch_bounds__(kFpThreads, NP * BB <= 2 ? 4 : 2)
           tok = 0;
         }
         const int64_t j = a.offE + (int64_t)tok * E + k;
-        const float d = pert(sw + (q / BB) * sw_stride, j, a.eps);
+        const float d = pert(sw, j, a.eps);
         const float th = a.theta[j];
         vp = th + d;
         vm = th - d;
       }
-      xin[q * E + k] = vp;
-      xin[NQ * E + q * E + k] = vm;
+      xin[b * E + k] = vp;
+      xin[BB * E + b * E + k] = vm;
     }
     __syncthreads();
     for (int l = 0; l < L; ++l) {
       const int in_l = l == 0 ? E : H;
-      const float* inp = l == 0 ? xin : hs + (l - 1) * 2 * NQ * H;
-      float* hl = hs + l * 2 * NQ * H;
-      float* cl = cs + l * 2 * NQ * H;
+      const float* inp = l == 0 ? xin : hs + (l - 1) * 2 * BB * H;
+      float* hl = hs + l * 2 * BB * H;
+      float* cl = cs + l * 2 * BB * H;
       if (VEC) {
-        build_tables<NQ>(inp, in_l, hl, H, U);
+        build_tables<BB>(inp, in_l, hl, H, U);
         __syncthreads();
       }
-      perturbed_gemv<NP, BB, VEC>(a, sw, sw_stride, a.offW[l], G4, in_l + H, in_l, inp, hl, U,
-                                  a.offB[l], gs, G4);
+      perturbed_gemv<BB, VEC>(a, sw, a.offW[l], G4, in_l + H, in_l, inp, hl, U, a.offB[l], gs, G4);
       __syncthreads();
-      for (int i = tid; i < 2 * NQ * H; i += nt) {
-        const int sq = i / H, u = i % H;
-        const float* G = gs + sq * G4;
+      for (int i = tid; i < 2 * BB * H; i += nt) {
+        const int sb = i / H, u = i % H;
+        const float* G = gs + sb * G4;
         const float ig = sigmoid_acc(G[u]);
         const float fg = sigmoid_acc(G[H + u]);
         const float gg = tanhf(G[2 * H + u]);
         const float og = sigmoid_acc(G[3 * H + u]);
-        const float c = fg * cl[sq * H + u] + ig * gg;
-        cl[sq * H + u] = c;
-        hl[sq * H + u] = og * tanhf(c);
+        const float c = fg * cl[sb * H + u] + ig * gg;
+        cl[sb * H + u] = c;
+        hl[sb * H + u] = og * tanhf(c);
       }
       __syncthreads();
     }
-    const float* htop = hs + (L - 1) * 2 * NQ * H;
+    const float* htop = hs + (L - 1) * 2 * BB * H;
     if (VEC) {
-      build_tables<NQ>(htop, H, htop, 0, U);
+      build_tables<BB>(htop, H, htop, 0, U);
       __syncthreads();
     }
-    perturbed_gemv<NP, BB, VEC>(a, sw, sw_stride, a.offWout, V, H, H, htop, htop, U, a.offBout,
-                                lg, V);
+    perturbed_gemv<BB, VEC>(a, sw, a.offWout, V, H, H, htop, htop, U, a.offBout, lg, V);
     __syncthreads();
-    for (int i = tid; i < 2 * NQ; i += nt) {
-      const int b = (i % NQ) % BB;
+    for (int i = tid; i < 2 * BB; i += nt) {
+      const int b = i % BB;
       if (b < nb) {
         int tg = a.targets[(int64_t)(r0 + b) * a.T + t];
         if (tg >= V || tg < -1) {
@@ -344,52 +313,46 @@ __global__ void __launch_bounds__(kFpThreads, NP * BB <= 2 ? 4 : 2)
     }
     __syncthreads();
   }
-  for (int i = tid; i < 2 * NQ; i += nt) {
-    const int s = i / NQ, q = i % NQ;
-    const int p = q / BB, b = q % BB;
-    if (b < nb && p < npv) a.rowloss[(int64_t)(2 * (pc + p) + s) * a.Bmax + r0 + b] = rl[i];
+  for (int i = tid; i < 2 * BB; i += nt) {
+    const int s = i / BB, b = i % BB;
+    if (b < nb) a.rowloss[(int64_t)(2 * ci + s) * a.Bmax + r0 + b] = rl[i];
   }
 }
 
-size_t fp32_smem_bytes(const zo_model_spec& s, int bb, int np, int64_t d_pad) {
+size_t fp32_smem_bytes(const zo_model_spec& s, int bb, int64_t d_pad) {
   const size_t E = s.embed, H = s.hidden, V = s.vocab, L = s.layers;
-  const size_t nq = (size_t)bb * np;
   const size_t gmax = ((E > H ? E : H) + H) / 4;   // groups of the widest step input
-  const size_t ufloats = (E % 4 == 0 && H % 4 == 0) ? 2 * nq * gmax * kUStride : 0;
-  return (size_t)np * (size_t)(d_pad / 8) +
-         sizeof(float) * (2 * nq * E + 4 * L * nq * H + 2 * nq * 4 * H + 2 * nq * V +
-                          ((2 * nq + 3) & ~3) + ufloats);
+  const size_t ufloats = (E % 4 == 0 && H % 4 == 0) ? 2 * bb * gmax * kUStride : 0;
+  return (size_t)(d_pad / 8) +
+         sizeof(float) * (2 * bb * E + 4 * L * bb * H + 2 * bb * 4 * H + 2 * bb * V +
+                          ((2 * bb + 3) & ~3) + ufloats);
 }
 
-template <int NP, int BB, bool VEC>
-static cudaError_t launch_fp32_cfg(const Fp32Args& a, size_t smem, cudaStream_t st) {
-  cudaFuncSetAttribute(fp32_forward_kernel<NP, BB, VEC>,
-                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+template <int BB, bool VEC>
+static cudaError_t launch_fp32_bb(const Fp32Args& a, int nprobe, size_t smem, cudaStream_t st) {
+  cudaFuncSetAttribute(fp32_forward_kernel<BB, VEC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       (int)smem);
   // ask for the largest shared-memory carveout so several CTAs share an SM
-  cudaFuncSetAttribute(fp32_forward_kernel<NP, BB, VEC>,
+  cudaFuncSetAttribute(fp32_forward_kernel<BB, VEC>,
                        cudaFuncAttributePreferredSharedMemoryCarveout, 100);
   int threads = 4 * a.H * 8 / 4;  // 8 lanes per row, 4 rows per warp
   threads = ((threads + 31) / 32) * 32;
   if (threads > kFpThreads) threads = kFpThreads;
   if (threads < 128) threads = 128;
-  dim3 grid((a.nprobe + NP - 1) / NP, (a.B + BB - 1) / BB);
-  fp32_forward_kernel<NP, BB, VEC><<<grid, threads, smem, st>>>(a);
+  dim3 grid(nprobe, (a.B + BB - 1) / BB);
+  fp32_forward_kernel<BB, VEC><<<grid, threads, smem, st>>>(a);
   count_launch();
   return cudaGetLastError();
 }
 
 template <bool VEC>
-static cudaError_t launch_fp32_vec(const Fp32Args& a, int bb, int np, size_t smem,
+static cudaError_t launch_fp32_vec(const Fp32Args& a, int bb, int nprobe, size_t smem,
                                    cudaStream_t st) {
-  if constexpr (VEC) {   // several probes per CTA only on the table path
-    if (np == 4) return launch_fp32_cfg<4, 1, VEC>(a, smem, st);
-    if (np == 2) return launch_fp32_cfg<2, 1, VEC>(a, smem, st);
-  }
   switch (bb) {
-    case 1: return launch_fp32_cfg<1, 1, VEC>(a, smem, st);
-    case 2: return launch_fp32_cfg<1, 2, VEC>(a, smem, st);
-    case 4: return launch_fp32_cfg<1, 4, VEC>(a, smem, st);
-    default: return launch_fp32_cfg<1, 8, VEC>(a, smem, st);
+    case 1: return launch_fp32_bb<1, VEC>(a, nprobe, smem, st);
+    case 2: return launch_fp32_bb<2, VEC>(a, nprobe, smem, st);
+    case 4: return launch_fp32_bb<4, VEC>(a, nprobe, smem, st);
+    default: return launch_fp32_bb<8, VEC>(a, nprobe, smem, st);
   }
 }
 
@@ -426,21 +389,9 @@ cudaError_t launch_fp32_forward(const zo_ctx* ctx, const float* theta, uint64_t 
   // leave SMs idle (a CTA's shared memory shrinks with its rows)
   int bb = ctx->fp32_bb;
   while (bb > 1 && (int64_t)nprobe * ((B + bb - 1) / bb) < ctx->sm_count) bb /= 2;
-  // probes per CTA (one batch row each): NP probes share every weight load
-  int np = 1;
-  if (vec && bb == 1) {
-    for (int cand = kFp32MaxProbes; cand > 1; cand /= 2) {
-      if (fp32_smem_bytes(ctx->spec, 1, cand, s.d_pad) <= kFp32SmemLimit &&
-          (int64_t)((nprobe + cand - 1) / cand) * B >= kFp32MinCtasPerSm * ctx->sm_count) {
-        np = cand;
-        break;
-      }
-    }
-  }
-  a.nprobe = nprobe;
-  const size_t smem = fp32_smem_bytes(ctx->spec, bb, np, s.d_pad);
-  return vec ? launch_fp32_vec<true>(a, bb, np, smem, st)
-             : launch_fp32_vec<false>(a, bb, np, smem, st);
+  const size_t smem = fp32_smem_bytes(ctx->spec, bb, s.d_pad);
+  return vec ? launch_fp32_vec<true>(a, bb, nprobe, smem, st)
+             : launch_fp32_vec<false>(a, bb, nprobe, smem, st);
 }
 
 }  // namespace zo

@@ -184,13 +184,13 @@ int zo_create(const zo_model_spec* spec, zo_ctx** out) {
     // (the probe's sign words for all d_pad parameters live in shared memory)
     const int64_t dp = c->seg.d_pad;
     int bb = 8;
-    while (bb > 1 && (bb / 2 >= B || fp32_smem_bytes(s, bb, 1, dp) > 200 * 1024)) bb /= 2;
-    if (fp32_smem_bytes(s, bb, 1, dp) > 200 * 1024) {
+    while (bb > 1 && (bb / 2 >= B || fp32_smem_bytes(s, bb, dp) > 200 * 1024)) bb /= 2;
+    if (fp32_smem_bytes(s, bb, dp) > 200 * 1024) {
       free_ctx(c);
       return ZO_ERR_UNSUPPORTED;
     }
     c->fp32_bb = bb;
-    c->fp32_smem = fp32_smem_bytes(s, bb, 1, dp);
+    c->fp32_smem = fp32_smem_bytes(s, bb, dp);
     // probe-column forward (several probes share each weight load) where the
     // shape and shared memory allow; it needs a transposed copy of W
     int64_t wt_floats = 0;

@@ -122,7 +122,7 @@ int fp32_wide_probes(const zo_model_spec& s, size_t limit, int64_t* wt_floats, s
 cudaError_t launch_fp32_wide(const zo_ctx* ctx, const float* theta, uint64_t seed, int probe0,
                              int nprobe, float eps, const int32_t* tokens, const int32_t* targets,
                              int B, int T, cudaStream_t st);
-// shared memory of the fp32 forward for bb batch rows x np probes per CTA
-size_t fp32_smem_bytes(const zo_model_spec& s, int bb, int np, int64_t d_pad);
+// shared memory of the per-probe fp32 forward for bb batch rows per CTA
+size_t fp32_smem_bytes(const zo_model_spec& s, int bb, int64_t d_pad);
 
 }  // namespace zo

@@ -71,11 +71,11 @@ extern "C" int zo_probe_losses_static(const zo_model_spec* spec, const float* th
   c.sm_count = g_sms[dev];
   zo::layout_of(c.spec, c.seg);
   int bb = 8;
-  while (bb > 1 && (bb / 2 >= batch || zo::fp32_smem_bytes(c.spec, bb, 1, c.seg.d_pad) > 200 * 1024))
+  while (bb > 1 && (bb / 2 >= batch || zo::fp32_smem_bytes(c.spec, bb, c.seg.d_pad) > 200 * 1024))
     bb /= 2;
-  if (zo::fp32_smem_bytes(c.spec, bb, 1, c.seg.d_pad) > 200 * 1024) return ZO_ERR_UNSUPPORTED;
+  if (zo::fp32_smem_bytes(c.spec, bb, c.seg.d_pad) > 200 * 1024) return ZO_ERR_UNSUPPORTED;
   c.fp32_bb = bb;
-  c.fp32_smem = zo::fp32_smem_bytes(c.spec, bb, 1, c.seg.d_pad);
+  c.fp32_smem = zo::fp32_smem_bytes(c.spec, bb, c.seg.d_pad);
   c.chunk = n_pert;
   c.rowloss = g_scratch_dev[dev];
   c.err = reinterpret_cast<unsigned*>(g_scratch_dev[dev] + ZO_STATIC_SCRATCH_FLOATS);
