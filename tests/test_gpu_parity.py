@@ -245,6 +245,24 @@ def test_token_out_of_range_is_reported():
         assert zo.zo_sync_status(ctx) == zo.ZO_OK   # cleared
 
 
+@pytest.mark.parametrize("t_bad", [0, 2])
+def test_token_out_of_range_is_reported_on_the_vocabulary_path(t_bad):
+    """bf16 model whose first layer takes its input term from the vocabulary
+    table: a bad token at t = 0 (first-step kernel) or later (cell epilogue)."""
+    V, E, H, L, B, T = 50, 512, 64, 1, 256, 3
+    cfg = W.small_config(vocab=V, embed=E, hidden=H, layers=L, dtype="bf16")
+    tok, tgt = W.random_batch(B, T, V, seed=1)
+    tok = tok.copy()
+    tok[7, t_bad] = V
+    with zo.Context(V, E, H, L, "bf16", B, T, 0) as ctx:
+        th = dev(W.init_theta(cfg))
+        lp = torch.empty(2, device="cuda")
+        lm = torch.empty(2, device="cuda")
+        zo.zo_probe_losses(ctx, th, 1, 2, 1e-3, dev(tok), dev(tgt), lp, lm)
+        assert zo.zo_sync_status(ctx) == zo.ZO_ERR_BOUNDS
+        assert zo.zo_sync_status(ctx) == zo.ZO_OK
+
+
 def test_nonfinite_loss_keeps_theta():
     cfg = W.CONFIGS["tiny"]
     theta = W.init_theta(cfg)
@@ -417,6 +435,12 @@ def test_probe_slices_match_full_call(name, slices):
     (2, 64, 64, 1, 1, 4, 2, 0, 0.0),        # V = 2, a single batch row
     (33, 64, 64, 2, 128, 1, 4, 0, 0.0),     # T = 1 (no recurrent input at all)
     (50, 64, 64, 1, 100, 3, 2, 0, 1.0),     # nothing scored: losses 0
+    # E >= 512 and >= 256 batch rows: layer 0's input term from the per-chunk
+    # vocabulary table (t = 0 from the table alone, later steps add it to the
+    # recurrent K stages in the epilogue)
+    (50, 512, 64, 2, 256, 3, 3, 0, 0.2),    # two layers, ignored targets
+    (64, 512, 128, 1, 300, 1, 2, 0, 0.0),   # T = 1: the first-step kernel only, ragged rows
+    (17, 1024, 64, 2, 260, 2, 3, 2, 0.3),   # two chunks, V = 17
 ])
 def test_bf16_edge_cases(V, E, H, L, B, T, n, chunk, frac):
     cfg = W.small_config(vocab=V, embed=E, hidden=H, layers=L, dtype="bf16")

@@ -53,6 +53,12 @@ struct CellArgs {
   float* raw;      // optional [P][Bmax][4H] pre-activations (then c, h are not written)
   unsigned* err;
   int gstride;     // rows between the four B boxes (H for the cell, BN/4 for the loss)
+  int kbeg;        // first K stage (the input stages are skipped when a vocabulary
+                   // table supplies the input term)
+  const float* vt; // vocabulary table [P][vtrows][4H] fp32 (layer 0), or null
+  int vtrows;
+  const int32_t* tokens;   // [B][T] (with vt)
+  int nobias;      // raw output without the bias (building the vocabulary table)
   // cross-entropy epilogue (MODE 1)
   int V, T, t;
   const int32_t* targets;  // [B][T]
@@ -321,7 +327,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       for (int64_t tile = blockIdx.x; tile < a.tiles && ok; tile += gridDim.x) {
         const TileCoord tc = decode_tile(a, tile, P);
         const int row0 = tc.m * 128 * MT;
-        for (int kb = 0; kb < a.nk; ++kb, ++it) {
+        for (int kb = a.kbeg; kb < a.nk; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1;
           if (!mbar_wait(empty_bar(s), ph ^ 1, abort_flag, a.err)) {
@@ -371,7 +377,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         tc_fence_after();
         const uint32_t dcol = tmem_base + ab * C::COLS;
-        for (int kb = 0; kb < a.nk; ++kb, ++it) {
+        for (int kb = a.kbeg; kb < a.nk; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1;
           if (!mbar_wait(ready_bar(s), ph, abort_flag, a.err)) {
@@ -387,7 +393,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             for (int mt = 0; mt < MT; ++mt) {
               const uint64_t adesc = umma_desc(sa + mt * C::A_SUB);
               umma_bf16(dcol + mt * BN, adesc + 2 * k16, bdesc + 2 * k16, idesc,
-                        (kb | k16) != 0 ? 1u : 0u);
+                        (kb != a.kbeg || k16 != 0) ? 1u : 0u);
             }
           }
           umma_commit(empty_bar(s));
@@ -425,7 +431,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       uint4 cw[RPT];
 #pragma unroll
       for (int rr = 0; rr < RPT; ++rr) cq[rr] = -1;
-      for (int kb = 0; kb < a.nk; ++kb, ++it) {
+      for (int kb = a.kbeg; kb < a.nk; ++kb, ++it) {
         const int s = it % STAGES;
         const uint32_t ph = (it / STAGES) & 1;
         if (!mbar_wait(full_bar(s), ph, abort_flag, a.err)) {
@@ -479,13 +485,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const int ab = tcount % ACC;
       const uint32_t aph = (tcount / ACC) & 1;
       if (MODE == 0 && !a.first && !a.raw) {
-        // while this tile's MMAs run, pull its c_{t-1} rows into L2 so the
-        // epilogue's loads hit L2 rather than HBM
+        // while this tile's MMAs run, pull its c_{t-1} rows (and the token's
+        // vocabulary-table rows) into L2 so the epilogue's loads hit L2
         for (int mt = 0; mt < MT; ++mt) {
           const int b = tc.m * 128 * MT + mt * 128 + rloc;
-          if (b < a.B)
+          if (b < a.B) {
             prefetch_l2(a.cst + ((int64_t)tc.ps * a.Bmax + b) * a.H + tc.n * C::U,
                         C::U * (int)sizeof(float));
+            if (a.vt) {
+              const int tok = a.tokens[(int64_t)b * a.T + a.t];
+              if (tok >= 0 && tok < a.V) {
+                const float* tr = a.vt + ((int64_t)tc.ps * a.vtrows + tok) * 4 * a.H + tc.n * C::U;
+#pragma unroll
+                for (int g = 0; g < 4; ++g) prefetch_l2(tr + g * a.H, C::U * (int)sizeof(float));
+              }
+            }
+          }
         }
       }
       if (!mbar_wait(accf_bar(ab), aph, abort_flag, a.err)) {
@@ -561,12 +576,29 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           if (live) {
             const int unit0 = tc.n * C::U + u0;
             float pre[4][8];
+            // input term from the vocabulary table (row of this batch row's token)
+            const float* trow = nullptr;
+            if (a.vt) {
+              int tok = a.tokens[(int64_t)b * a.T + a.t];
+              if (tok < 0 || tok >= a.V) {
+                latch(a.err, kErrBounds);
+                tok = 0;
+              }
+              trow = a.vt + ((int64_t)tc.ps * a.vtrows + tok) * 4 * a.H + unit0;
+            }
 #pragma unroll
             for (int g = 0; g < 4; ++g) {
               const float4* bp = reinterpret_cast<const float4*>(bias + g * a.H + unit0);
 #pragma unroll
               for (int q4 = 0; q4 < 2; ++q4) {
-                const float4 bv = __ldg(bp + q4);
+                float4 bv = a.nobias ? make_float4(0.f, 0.f, 0.f, 0.f) : __ldg(bp + q4);
+                if (trow) {
+                  const float4 tv = __ldg(reinterpret_cast<const float4*>(trow + g * a.H) + q4);
+                  bv.x += tv.x;
+                  bv.y += tv.y;
+                  bv.z += tv.z;
+                  bv.w += tv.w;
+                }
                 pre[g][4 * q4 + 0] = __uint_as_float(acc[g][4 * q4 + 0]) + bv.x;
                 pre[g][4 * q4 + 1] = __uint_as_float(acc[g][4 * q4 + 1]) + bv.y;
                 pre[g][4 * q4 + 2] = __uint_as_float(acc[g][4 * q4 + 2]) + bv.z;
@@ -705,16 +737,26 @@ static cudaError_t launch_cfg(const CUtensorMap& A0, const CUtensorMap& A1, cons
 }
 
 cudaError_t launch_cell_tc(const zo_ctx* ctx, int layer, int t, int B, int nprobe, int probe0,
-                           uint64_t seed, float eps, float* raw_out, cudaStream_t st) {
+                           uint64_t seed, float eps, float* raw_out, const int32_t* tokens, int T,
+                           bool vocab, cudaStream_t st) {
   const zo_model_spec& s = ctx->spec;
   const int H = s.hidden, E = s.embed;
   const int P = 2 * nprobe;
   const int K0 = layer == 0 ? E : H;
+  // with the vocabulary table, layer 0 runs only its recurrent K stages (none
+  // at t = 0: that step is launch_vocab_first)
+  const bool tab = vocab && layer == 0;
+  if (tab && (t == 0 || !ctx->vt)) return cudaErrorInvalidValue;
   CellArgs a;
   a.K0 = K0;
   a.H = H;
   a.Ktot = K0 + H;
   a.nk = (t == 0 ? K0 : K0 + H) / 64;
+  a.kbeg = tab ? K0 / 64 : 0;
+  a.vt = tab ? ctx->vt : nullptr;
+  a.vtrows = kVocabRows;
+  a.tokens = tokens;
+  a.nobias = 0;
   a.B = B;
   a.Bmax = s.max_batch;
   a.group = 8;
@@ -732,7 +774,7 @@ cudaError_t launch_cell_tc(const zo_ctx* ctx, int layer, int t, int B, int nprob
   a.raw = raw_out;
   a.err = ctx->err;
   a.V = s.vocab;
-  a.T = 0;
+  a.T = T;
   a.t = t;
   a.targets = nullptr;
   a.rowloss = nullptr;
@@ -775,6 +817,11 @@ cudaError_t launch_loss_tc(const zo_ctx* ctx, const int32_t* targets, int t, int
   a.raw = nullptr;
   a.err = ctx->err;
   a.gstride = 16;
+  a.kbeg = 0;
+  a.vt = nullptr;
+  a.vtrows = 0;
+  a.tokens = nullptr;
+  a.nobias = 0;
   a.V = s.vocab;
   a.T = T;
   a.t = t;
@@ -783,6 +830,52 @@ cudaError_t launch_loss_tc(const zo_ctx* ctx, const int32_t* targets, int t, int
   const CellMaps& m = *ctx->maps;
   const CUtensorMap& A0 = m.h[L - 1][t & 1];
   return launch_cfg<2, 64, 4, 2, 1>(A0, A0, m.wout, a, P, ctx->sm_count, st);
+}
+
+// Vocabulary table of layer 0's input term for the chunk's probe-signs:
+// vt[ps][v][:] = E'_ps[v] (W_0x +- eps P)^T, E'_ps the perturbed embedding in
+// bf16, W_0x the first E columns of W_0 perturbed in shared memory as in every
+// cell launch; the same mainloop with the vocabulary rows as the batch, the
+// input K stages only, and the raw fp32 accumulators (no bias) as output.
+cudaError_t launch_vocab_table(const zo_ctx* ctx, int nprobe, int probe0, uint64_t seed, float eps,
+                               cudaStream_t st) {
+  const zo_model_spec& s = ctx->spec;
+  if (!ctx->vt) return cudaErrorInvalidValue;
+  const int H = s.hidden, E = s.embed;
+  const int P = 2 * nprobe;
+  CellArgs a;
+  a.K0 = E;
+  a.H = H;
+  a.Ktot = E + H;
+  a.nk = E / 64;
+  a.kbeg = 0;
+  a.vt = nullptr;
+  a.vtrows = kVocabRows;
+  a.tokens = nullptr;
+  a.nobias = 1;
+  a.B = s.vocab;             // live rows: the vocabulary
+  a.Bmax = kVocabRows;       // row stride of the raw output
+  a.group = 8;
+  a.seed = seed;
+  a.probe0 = probe0;
+  a.eps = eps;
+  a.offW = ctx->seg.off[ctx->seg.W[0]];
+  a.small_p = ctx->small_p;
+  a.sstride = ctx->small.stride;
+  a.soffb = ctx->small.b[0];
+  a.cst = nullptr;
+  a.hout = nullptr;
+  a.first = 1;
+  a.raw = ctx->vt;
+  a.err = ctx->err;
+  a.V = s.vocab;
+  a.T = 0;
+  a.t = 0;
+  a.targets = nullptr;
+  a.rowloss = nullptr;
+  a.gstride = H;
+  const CellMaps& m = *ctx->maps;
+  return launch_cfg<2, 256, 3, 1, 0>(m.x, m.x, m.w[0], a, P, ctx->sm_count, st);
 }
 
 }  // namespace zo

@@ -92,6 +92,94 @@ cudaError_t launch_perturb_small(const zo_ctx* ctx, const float* theta, uint64_t
 }
 
 // ---------------------------------------------------------------------------
+// Vocabulary rows of the first layer's input: x[ps][v][:] = bf16(E'_ps[v][:])
+// for every token v (the A operand of the vocabulary-table launch).
+// ---------------------------------------------------------------------------
+__global__ void vocab_x_kernel(const float* __restrict__ small_p, int64_t stride, int64_t offE,
+                               int Bmax, int E, int V, int P, __nv_bfloat16* __restrict__ x) {
+  const int e2 = E / 2;
+  const int64_t total = (int64_t)P * V * e2;
+  for (int64_t k = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; k < total;
+       k += (int64_t)gridDim.x * blockDim.x) {
+    const int c = (int)(k % e2);
+    const int64_t pv = k / e2;
+    const int v = (int)(pv % V);
+    const int ps = (int)(pv / V);
+    const float2 u =
+        reinterpret_cast<const float2*>(small_p + ps * stride + offE + (int64_t)v * E)[c];
+    reinterpret_cast<__nv_bfloat162*>(x + ((int64_t)ps * Bmax + v) * E)[c] =
+        __floats2bfloat162_rn(u.x, u.y);
+  }
+}
+
+// The cell epilogue's approximations (tanh.approx), so that t = 0 from the
+// vocabulary table matches what the tensor-core epilogue computes.
+__device__ __forceinline__ float tanh_ap(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float sigmoid_ap(float x) { return fmaf(0.5f, tanh_ap(0.5f * x), 0.5f); }
+
+// Layer 0 at t = 0 from the vocabulary table: h_{-1} = c_{-1} = 0, so the
+// pre-activations are the table row of the token plus the bias.
+__global__ void vocab_first_kernel(const float* __restrict__ vt, int vtrows,
+                                   const float* __restrict__ small_p, int64_t stride,
+                                   int64_t offb, const int32_t* __restrict__ tokens, int T, int B,
+                                   int Bmax, int H, int V, int P, float* __restrict__ cst,
+                                   __nv_bfloat16* __restrict__ hout, unsigned* err) {
+  const int64_t total = (int64_t)P * B * H;
+  for (int64_t k = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; k < total;
+       k += (int64_t)gridDim.x * blockDim.x) {
+    const int u = (int)(k % H);
+    const int64_t pb = k / H;
+    const int b = (int)(pb % B);
+    const int ps = (int)(pb / B);
+    int tok = tokens[(int64_t)b * T];
+    if (tok < 0 || tok >= V) {
+      latch(err, kErrBounds);
+      tok = 0;
+    }
+    const float* tr = vt + ((int64_t)ps * vtrows + tok) * 4 * H;
+    const float* bias = small_p + ps * stride + offb;
+    const float ig = sigmoid_ap(tr[u] + bias[u]);
+    const float gg = tanh_ap(tr[2 * H + u] + bias[2 * H + u]);
+    const float og = sigmoid_ap(tr[3 * H + u] + bias[3 * H + u]);
+    const float c = ig * gg;
+    const int64_t o = ((int64_t)ps * Bmax + b) * H + u;
+    cst[o] = c;
+    hout[o] = __float2bfloat16_rn(og * tanh_ap(c));
+  }
+}
+
+cudaError_t launch_vocab_first(const zo_ctx* ctx, const int32_t* tokens, int B, int T, int nprobe,
+                               cudaStream_t st) {
+  const zo_model_spec& s = ctx->spec;
+  const int P = 2 * nprobe, H = s.hidden;
+  const int64_t total = (int64_t)P * B * H;
+  int64_t grid = (total + 255) / 256;
+  if (grid > (int64_t)ctx->sm_count * 16) grid = (int64_t)ctx->sm_count * 16;
+  vocab_first_kernel<<<(int)grid, 256, 0, st>>>(ctx->vt, kVocabRows, ctx->small_p,
+                                                ctx->small.stride, ctx->small.b[0], tokens, T, B,
+                                                s.max_batch, H, s.vocab, P, ctx->cst,
+                                                ctx->h /* layer 0, parity of t = 0 */, ctx->err);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_vocab_x(const zo_ctx* ctx, int nprobe, cudaStream_t st) {
+  const zo_model_spec& s = ctx->spec;
+  const int P = 2 * nprobe;
+  const int64_t total = (int64_t)P * s.vocab * (s.embed / 2);
+  int64_t grid = (total + 255) / 256;
+  if (grid > (int64_t)ctx->sm_count * 16) grid = (int64_t)ctx->sm_count * 16;
+  vocab_x_kernel<<<(int)grid, 256, 0, st>>>(ctx->small_p, ctx->small.stride, ctx->small.E,
+                                            s.max_batch, s.embed, s.vocab, P, ctx->x);
+  count_launch();
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
 // x_t[ps][b][:] = bf16(E_perturbed[ps][token[b, t]][:])  (first layer input)
 // ---------------------------------------------------------------------------
 __global__ void gather_x_kernel(const float* __restrict__ small_p, int64_t stride, int64_t offE,

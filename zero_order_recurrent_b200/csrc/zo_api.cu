@@ -101,6 +101,7 @@ void free_ctx(zo_ctx* c) {
   cudaFree(c->lm);
   cudaFree(c->coef);
   cudaFree(c->wt);
+  cudaFree(c->vt);
   for (auto& r : c->prof) {
     if (r.a) cudaEventDestroy(r.a);
     if (r.b) cudaEventDestroy(r.b);
@@ -216,7 +217,13 @@ int zo_create(const zo_model_spec* spec, zo_ctx** out) {
     sl.bout = o;
     o += align4(V);
     sl.stride = o;
-    const int64_t per_ps = 2 * B * E + L * 2 * B * H * 2 + L * B * H * 4 + sl.stride * 4 + B * 4;
+    // the first layer's input term from a per-chunk vocabulary table where the
+    // embedding is wide enough that the table's gather (16 B per gate row and
+    // batch row) costs less than the input K stages it replaces (2 E flops),
+    // and the vocabulary rows fit one 256-row tile of the x buffer
+    c->vocab = E >= 512 && B >= 256;
+    const int64_t per_ps = 2 * B * E + L * 2 * B * H * 2 + L * B * H * 4 + sl.stride * 4 + B * 4 +
+                           (c->vocab ? (int64_t)kVocabRows * 4 * H * 4 : 0);
     int chunk = s.chunk;
     if (chunk == 0) {
       size_t fr = 0, tot = 0;
@@ -233,6 +240,7 @@ int zo_create(const zo_model_spec* spec, zo_ctx** out) {
     alloc((void**)&c->h, sizeof(__nv_bfloat16) * L * 2 * P * B * H);
     alloc((void**)&c->cst, sizeof(float) * L * P * B * H);
     alloc((void**)&c->rowloss, sizeof(float) * P * B);
+    if (c->vocab) alloc((void**)&c->vt, sizeof(float) * P * kVocabRows * 4 * H);
     if (rc == ZO_OK && !make_cell_maps(c)) rc = ZO_ERR_CUDA;
   }
   if (rc == ZO_OK && cudaDeviceSynchronize() != cudaSuccess) rc = ZO_ERR_CUDA;
@@ -328,14 +336,31 @@ static int probe_losses_range(zo_ctx* ctx, const float* theta, uint64_t seed, in
     ZO_CUDA(timed(ctx, st, ZO_KIND_OTHER, 0.0, 0.0,
                   [&] { return launch_perturb_small(ctx, theta, seed, probe_begin + p0, np, eps, st); }));
     ZO_CUDA(cudaMemsetAsync(ctx->rowloss, 0, sizeof(float) * 2 * np * ctx->spec.max_batch, st));
+    const bool vocab = ctx->vocab;
+    if (vocab) {
+      // executed flops: the 256-row tile over the vocabulary rows
+      const double fl = 2.0 * P * 256.0 * Ee * 4.0 * Hh;
+      ZO_CUDA(timed(ctx, st, ZO_KIND_OTHER, 0.0, 0.0, [&] { return launch_vocab_x(ctx, np, st); }));
+      ZO_CUDA(timed(ctx, st, ZO_KIND_CELL, fl, 0.0, [&] {
+        return launch_vocab_table(ctx, np, probe_begin + p0, seed, eps, st);
+      }));
+    }
     for (int t = 0; t < T; ++t) {
-      ZO_CUDA(timed(ctx, st, ZO_KIND_OTHER, 0.0, P * B * Ee * 2.0,
-                    [&] { return launch_gather_x(ctx, tokens, t, B, T, np, st); }));
+      if (!vocab)
+        ZO_CUDA(timed(ctx, st, ZO_KIND_OTHER, 0.0, P * B * Ee * 2.0,
+                      [&] { return launch_gather_x(ctx, tokens, t, B, T, np, st); }));
       for (int l = 0; l < L; ++l) {
-        const double Krun = (double)(l == 0 ? Ee : Hh) + (t == 0 ? 0.0 : (double)Hh);
+        if (vocab && l == 0 && t == 0) {
+          ZO_CUDA(timed(ctx, st, ZO_KIND_OTHER, 0.0, 0.0,
+                        [&] { return launch_vocab_first(ctx, tokens, B, T, np, st); }));
+          continue;
+        }
+        const double Kin = (vocab && l == 0) ? 0.0 : (double)(l == 0 ? Ee : Hh);
+        const double Krun = Kin + (t == 0 ? 0.0 : (double)Hh);
         const double fl = 2.0 * P * B * Krun * 4.0 * Hh;
         ZO_CUDA(timed(ctx, st, ZO_KIND_CELL, fl, 0.0, [&] {
-          return launch_cell_tc(ctx, l, t, B, np, probe_begin + p0, seed, eps, nullptr, st);
+          return launch_cell_tc(ctx, l, t, B, np, probe_begin + p0, seed, eps, nullptr, tokens, T,
+                                vocab, st);
         }));
       }
       ZO_CUDA(timed(ctx, st, ZO_KIND_LOSS, 2.0 * P * B * Hh * Vv, P * B * Hh * 2.0, [&] {
@@ -500,7 +525,8 @@ int zo_debug_cell_preact(zo_ctx* ctx, const float* theta, uint64_t seed, int32_t
   ctx->shadow_fresh = true;
   ZO_CUDA(launch_perturb_small(ctx, theta, seed, probe0, n_probes, eps, st));
   ZO_CUDA(launch_gather_x(ctx, tokens, 0, batch, seq, n_probes, st));
-  ZO_CUDA(launch_cell_tc(ctx, 0, 0, batch, n_probes, probe0, seed, eps, preact, st));
+  ZO_CUDA(launch_cell_tc(ctx, 0, 0, batch, n_probes, probe0, seed, eps, preact, tokens, seq, false,
+                         st));
   return ZO_OK;
 }
 

@@ -66,6 +66,10 @@ struct zo_ctx {
   __nv_bfloat16* h = nullptr;    // [L][2][2*chunk][B][H]
   float* cst = nullptr;          // [L][2*chunk][B][H]
   zo::CellMaps* maps = nullptr;  // host copy of the tensor maps
+  // vocabulary table of the first layer's input term (bf16 path, wide
+  // embeddings): vt[ps][v][4H] = E'_ps[v] (W_0x +- eps P)^T, built once per chunk
+  float* vt = nullptr;
+  bool vocab = false;
   // both paths
   float* rowloss = nullptr;      // [2*chunk][B]
   // zo_step_host staging (device)
@@ -113,7 +117,16 @@ cudaError_t launch_gather_x(const zo_ctx* ctx, const int32_t* tokens, int t, int
 cudaError_t launch_loss_tc(const zo_ctx* ctx, const int32_t* targets, int t, int B, int T,
                            int nprobe, int probe0, uint64_t seed, float eps, cudaStream_t st);
 cudaError_t launch_cell_tc(const zo_ctx* ctx, int layer, int t, int B, int nprobe, int probe0,
-                           uint64_t seed, float eps, float* raw_out, cudaStream_t st);
+                           uint64_t seed, float eps, float* raw_out, const int32_t* tokens, int T,
+                           bool vocab, cudaStream_t st);
+// vocabulary table (rows kVocabRows per probe-sign) and the first step of
+// layer 0 from it
+constexpr int kVocabRows = 64;
+cudaError_t launch_vocab_table(const zo_ctx* ctx, int nprobe, int probe0, uint64_t seed, float eps,
+                               cudaStream_t st);
+cudaError_t launch_vocab_first(const zo_ctx* ctx, const int32_t* tokens, int B, int T, int nprobe,
+                               cudaStream_t st);
+cudaError_t launch_vocab_x(const zo_ctx* ctx, int nprobe, cudaStream_t st);
 bool make_cell_maps(zo_ctx* ctx);
 void layout_of(const zo_model_spec& sp, Segments& s);
 // probe-column fp32 forward: probes per CTA that fit `limit` bytes of shared
