@@ -52,6 +52,8 @@ CONFIGS = {
     "charlm": Config("charlm", 50, 256, 1024, 2, "bf16", 1024, 10, 64, 1e-3, 1e-3, "markov"),
     "lstm270m": Config("lstm270m", 50, 4096, 4096, 2, "bf16", 1024, 10, 32, 1e-3, 1e-3, "markov"),
     "lstm1b": Config("lstm1b", 50, 8192, 8192, 2, "bf16", 1024, 10, 16, 1e-3, 1e-3, "markov", 16),
+    # the pages' single-device feasibility scale (~4.3B parameters, 17 GB fp32)
+    "lstm4b": Config("lstm4b", 50, 16384, 16384, 2, "bf16", 1024, 10, 16, 1e-3, 1e-3, "markov", 16),
 }
 
 INIT_SEED = 1

@@ -58,7 +58,6 @@ struct CellArgs {
   const float* vt; // vocabulary table [P][vtrows][4H] fp32 (layer 0), or null
   int vtrows;
   const int32_t* tokens;   // [B][T] (with vt)
-  int nobias;      // raw output without the bias (building the vocabulary table)
   // cross-entropy epilogue (MODE 1)
   int V, T, t;
   const int32_t* targets;  // [B][T]
@@ -263,6 +262,9 @@ struct TcCfg {
   static_assert(TMEM_COLS == 128 || TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM columns");
 };
 
+// MODE 0: cell step.  1: output projection + cross-entropy.  2: cell step of
+// layer 0 whose input term comes from the vocabulary table (added in the
+// epilogue).  3: the vocabulary table itself (raw accumulators, no bias).
 template <int MT, int BN, int STAGES, int ACC, int MODE>
 __global__ void __launch_bounds__(kTcThreads, 1)
     cell_tc_kernel(const __grid_constant__ CUtensorMap mapA0, const __grid_constant__ CUtensorMap mapA1,
@@ -484,7 +486,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const TileCoord tc = decode_tile(a, tile, P);
       const int ab = tcount % ACC;
       const uint32_t aph = (tcount / ACC) & 1;
-      if (MODE == 0 && !a.first && !a.raw) {
+      if ((MODE == 0 || MODE == 2) && !a.first && !a.raw) {
         // while this tile's MMAs run, pull its c_{t-1} rows (and the token's
         // vocabulary-table rows) into L2 so the epilogue's loads hit L2
         for (int mt = 0; mt < MT; ++mt) {
@@ -492,7 +494,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           if (b < a.B) {
             prefetch_l2(a.cst + ((int64_t)tc.ps * a.Bmax + b) * a.H + tc.n * C::U,
                         C::U * (int)sizeof(float));
-            if (a.vt) {
+            if constexpr (MODE == 2) {
               const int tok = a.tokens[(int64_t)b * a.T + a.t];
               if (tok >= 0 && tok < a.V) {
                 const float* tr = a.vt + ((int64_t)tc.ps * a.vtrows + tok) * 4 * a.H + tc.n * C::U;
@@ -578,7 +580,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             float pre[4][8];
             // input term from the vocabulary table (row of this batch row's token)
             const float* trow = nullptr;
-            if (a.vt) {
+            if constexpr (MODE == 2) {
               int tok = a.tokens[(int64_t)b * a.T + a.t];
               if (tok < 0 || tok >= a.V) {
                 latch(a.err, kErrBounds);
@@ -591,8 +593,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               const float4* bp = reinterpret_cast<const float4*>(bias + g * a.H + unit0);
 #pragma unroll
               for (int q4 = 0; q4 < 2; ++q4) {
-                float4 bv = a.nobias ? make_float4(0.f, 0.f, 0.f, 0.f) : __ldg(bp + q4);
-                if (trow) {
+                float4 bv = MODE == 3 ? make_float4(0.f, 0.f, 0.f, 0.f) : __ldg(bp + q4);
+                if constexpr (MODE == 2) {
                   const float4 tv = __ldg(reinterpret_cast<const float4*>(trow + g * a.H) + q4);
                   bv.x += tv.x;
                   bv.y += tv.y;
@@ -726,7 +728,7 @@ static cudaError_t launch_cfg(const CUtensorMap& A0, const CUtensorMap& A1, cons
                               CellArgs a, int P, int sms, cudaStream_t st) {
   using C = TcCfg<MT, BN, STAGES, ACC>;
   a.m_tiles = (a.B + 128 * MT - 1) / (128 * MT);
-  a.n_tiles = MODE == 0 ? a.H / C::U : 1;
+  a.n_tiles = MODE != 1 ? a.H / C::U : 1;
   a.tiles = (int64_t)P * a.m_tiles * a.n_tiles;
   cudaFuncSetAttribute(cell_tc_kernel<MT, BN, STAGES, ACC, MODE>,
                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
@@ -756,7 +758,6 @@ cudaError_t launch_cell_tc(const zo_ctx* ctx, int layer, int t, int B, int nprob
   a.vt = tab ? ctx->vt : nullptr;
   a.vtrows = kVocabRows;
   a.tokens = tokens;
-  a.nobias = 0;
   a.B = B;
   a.Bmax = s.max_batch;
   a.group = 8;
@@ -784,6 +785,7 @@ cudaError_t launch_cell_tc(const zo_ctx* ctx, int layer, int t, int B, int nprob
   a.gstride = H;
   // 256 batch rows x 256 gate rows per tile (all 512 TMEM columns): the
   // fastest shape measured for every model size here (K from 1280 to 16384)
+  if (tab) return launch_cfg<2, 256, 3, 1, 2>(A0, A1, m.w[layer], a, P, ctx->sm_count, st);
   return launch_cfg<2, 256, 3, 1, 0>(A0, A1, m.w[layer], a, P, ctx->sm_count, st);
 }
 
@@ -821,7 +823,6 @@ cudaError_t launch_loss_tc(const zo_ctx* ctx, const int32_t* targets, int t, int
   a.vt = nullptr;
   a.vtrows = 0;
   a.tokens = nullptr;
-  a.nobias = 0;
   a.V = s.vocab;
   a.T = T;
   a.t = t;
@@ -852,7 +853,6 @@ cudaError_t launch_vocab_table(const zo_ctx* ctx, int nprobe, int probe0, uint64
   a.vt = nullptr;
   a.vtrows = kVocabRows;
   a.tokens = nullptr;
-  a.nobias = 1;
   a.B = s.vocab;             // live rows: the vocabulary
   a.Bmax = kVocabRows;       // row stride of the raw output
   a.group = 8;
@@ -875,7 +875,7 @@ cudaError_t launch_vocab_table(const zo_ctx* ctx, int nprobe, int probe0, uint64
   a.rowloss = nullptr;
   a.gstride = H;
   const CellMaps& m = *ctx->maps;
-  return launch_cfg<2, 256, 3, 1, 0>(m.x, m.x, m.w[0], a, P, ctx->sm_count, st);
+  return launch_cfg<2, 256, 3, 1, 3>(m.x, m.x, m.w[0], a, P, ctx->sm_count, st);
 }
 
 }  // namespace zo
