@@ -18,7 +18,7 @@ Zero-Order Optimization", Chaubard & Kochenderfer, arXiv 2505.17852):
   formula when eta = eps.
 * pith.science review, "Assumptions": E[p] = 0 and E[p p^T] = I.
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings where the pages are silent:
 
 1. Model: textbook LSTM, gate blocks in the order i, f, g, o, one bias per
    layer, h0 = c0 = 0, no forget-gate offset; token embedding in front and a

@@ -183,7 +183,7 @@ def _all_signs(d):
 
 
 def test_quadratic_all_sign_vectors_give_exact_gradient():
-    """The benchmark spec test 1: on L = 1/2 x^T A x + b^T x + k, averaging the central
+    """Method check 1 (exactness): on L = 1/2 x^T A x + b^T x + k, averaging the central
     difference over all 2^d Rademacher vectors returns the gradient exactly
     (the cubic remainder vanishes and sum_p p p^T = 2^d I).  With eta = eps the
     update is theta' = theta - eps * grad."""
@@ -246,7 +246,7 @@ def test_app_c_antithetic_forward_difference_equals_central_difference():
 
 
 def test_antisymmetry_negated_probe_negates_coefficient():
-    """The benchmark spec test 2: replacing p_i by -p_i swaps L+ and L-, so c_i -> -c_i
+    """Method check 2 (antisymmetry): replacing p_i by -p_i swaps L+ and L-, so c_i -> -c_i
     exactly (IEEE subtraction is antisymmetric)."""
     cfg = W.CONFIGS["tiny"]
     spec = (cfg.vocab, cfg.embed, cfg.hidden, cfg.layers)
@@ -328,7 +328,7 @@ def test_coordinate_cd_matches_autograd():
 
 
 def test_estimator_converges_to_coordinate_cd_gradient():
-    """The benchmark spec test 3: with K >> d probes, g_hat_K (Philox probes, oracle
+    """Method check 3 (convergence): with K >> d probes, g_hat_K (Philox probes, oracle
     losses) approaches the coordinate CD gradient; for Rademacher probes
     E cos ~ sqrt(K / (K + d - 1))."""
     cfg = W.small_config(vocab=3, embed=2, hidden=2, layers=1)
