@@ -517,11 +517,15 @@ cudaError_t launch_fp32_wide(const zo_ctx* ctx, const float* theta, uint64_t see
   a.small_words = P.small_words;
   a.gmax = P.gmax;
   a.rmax = P.rmax;
-  a.pmax = partial_floats(P, L, 2 * ctx->fp32_wide_np);
+  // four probes per CTA share each weight load best; with few probes (a slice
+  // of a probe-parallel step, small tests) two per CTA keep more SMs busy
+  int np = ctx->fp32_wide_np;
+  if (np == 4 && (int64_t)((nprobe + 3) / 4) * B < (int64_t)ctx->sm_count * 3 / 4) np = 2;
+  a.pmax = partial_floats(P, L, 2 * np);
   a.rowloss = ctx->rowloss;
   a.err = ctx->err;
-  const size_t smem = wide_smem(sp, P, ctx->fp32_wide_np);
-  return ctx->fp32_wide_np == 4 ? launch_wide_np<4>(a, smem, st) : launch_wide_np<2>(a, smem, st);
+  const size_t smem = wide_smem(sp, P, np);
+  return np == 4 ? launch_wide_np<4>(a, smem, st) : launch_wide_np<2>(a, smem, st);
 }
 
 }  // namespace zo
