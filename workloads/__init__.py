@@ -138,6 +138,54 @@ def copy_batch(batch: int = 8, length: int = 10, seed: int = 0):
     return tokens, targets
 
 
+def task_length(task: str, length: int) -> int:
+    """Positions of one example of a transduction task with `length` data digits."""
+    return 3 * length + 3 if task == "add" else 2 * length + 1
+
+
+def transduction_batch(task: str, lengths, T: int, seed: int = 0):
+    """One batch of a transduction task (the pages' COPY / REVERSE / ADD
+    workloads; they give the lengths only, the formats are readings), each row
+    padded with blanks (token 0, target -1) to T positions.
+
+    Tokens: data digits 1..8, delimiter 9, blank 0; target -1 = not scored.
+      copy:    x_1..x_L, 9, 0 x L        -> targets -1 x (L+1), x_1..x_L
+      reverse: x_1..x_L, 9, 0 x L        -> targets -1 x (L+1), x_L..x_1
+      add:     a_1..a_L, 9, b_1..b_L, 9, 0 x (L+1)  (base-8 digits, least
+               significant first, token = digit + 1)
+               -> targets -1 x (2L+2), then the L+1 digits of a + b
+    """
+    rng = np.random.default_rng(seed)
+    lengths = np.asarray(lengths, dtype=np.int64)
+    B = len(lengths)
+    tokens = np.zeros((B, T), dtype=np.int32)
+    targets = np.full((B, T), -1, dtype=np.int32)
+    for r, L in enumerate(lengths):
+        L = int(L)
+        if task_length(task, L) > T:
+            raise ValueError(f"{task} of length {L} needs {task_length(task, L)} > {T} positions")
+        if task in ("copy", "reverse"):
+            x = rng.integers(1, 9, size=L, dtype=np.int32)
+            tokens[r, :L] = x
+            tokens[r, L] = 9
+            targets[r, L + 1:2 * L + 1] = x if task == "copy" else x[::-1]
+        elif task == "add":
+            a = rng.integers(0, 8, size=L)
+            b = rng.integers(0, 8, size=L)
+            tokens[r, :L] = a + 1
+            tokens[r, L] = 9
+            tokens[r, L + 1:2 * L + 1] = b + 1
+            tokens[r, 2 * L + 1] = 9
+            carry = 0
+            for i in range(L + 1):
+                s = carry + (int(a[i]) + int(b[i]) if i < L else 0)
+                targets[r, 2 * L + 2 + i] = s % 8 + 1
+                carry = s // 8
+        else:
+            raise ValueError(f"unknown task {task}")
+    return tokens, targets
+
+
 def overfit_batch(vocab: int = 50, length: int = 100, seed: int = 0):
     """One uniform random sequence of length+1 tokens, batch 1."""
     rng = np.random.default_rng(seed)
