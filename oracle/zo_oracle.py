@@ -272,6 +272,18 @@ def coefficients(loss_plus, loss_minus, n_pert: int, eps: float, eta: float) -> 
     return h * (lp - lm) / (2.0 * e * n_pert)
 
 
+def coefficients_forward(loss_plus, loss0, n_pert: int, eps: float, eta: float) -> np.ndarray:
+    """Forward-difference coefficients c_i = eta * (L+_i - L0) / (eps n_pert),
+    L0 = L(theta): the one-sided estimator g_hat = 1/n sum_i (L(theta + eps u_i)
+    - L(theta))/eps u_i.  Over an antithetic set {u_i, -u_i} it equals the
+    central difference (pith.science review, "Circularity Check": the
+    Appendix C identity)."""
+    lp = np.asarray(loss_plus, dtype=np.float64)
+    e = float(np.float32(eps))
+    h = float(np.float32(eta))
+    return h * (lp - float(loss0)) / (e * n_pert)
+
+
 def update_with_probes(theta, probes: np.ndarray, coeffs) -> np.ndarray:
     """theta' = theta - sum_i c_i p_i with explicit probe vectors [n, d]."""
     th = np.asarray(theta, dtype=np.float64)

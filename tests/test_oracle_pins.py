@@ -245,6 +245,26 @@ def test_app_c_antithetic_forward_difference_equals_central_difference():
     assert np.allclose(fd, cd, rtol=1e-9, atol=1e-12)
 
 
+def test_forward_coefficients_over_antithetic_set_give_the_central_update():
+    """Forward-difference coefficients (eta (L+ - L0)/(eps n)) over the
+    antithetic set {p_i, -p_i} (n = 2K; L(theta - eps p_i) is the + loss of
+    -p_i) move theta exactly as the central coefficients over {p_i} (n = K):
+    the Appendix C identity on the coefficients.  Plus one value by hand."""
+    assert O.coefficients_forward([3.0], 2.0, 2, 0.5, 0.25)[0] == 0.25
+    cfg = W.small_config(vocab=5, embed=3, hidden=4, layers=1)
+    spec = (cfg.vocab, cfg.embed, cfg.hidden, cfg.layers)
+    theta = W.init_theta(cfg, seed=2)
+    tok, tgt = W.random_batch(3, 5, cfg.vocab, seed=1)
+    seed, K, eps, eta = W.step_seed(6), 5, 1e-3, 3e-2
+    lp, lm = O.probe_losses(theta, spec, seed, K, eps, tok, tgt)
+    l0 = O.loss_at(theta, spec, tok, tgt)
+    P = O.probe_matrix(spec, seed, K).astype(np.float64)
+    cf = O.coefficients_forward(np.concatenate([lp, lm]), l0, 2 * K, eps, eta)
+    fwd = cf[:K] @ P + cf[K:] @ (-P)
+    cen = O.coefficients(lp, lm, K, eps, eta) @ P
+    assert np.allclose(fwd, cen, rtol=1e-12, atol=1e-15)
+
+
 def test_antisymmetry_negated_probe_negates_coefficient():
     """Method check 2 (antisymmetry): replacing p_i by -p_i swaps L+ and L-, so c_i -> -c_i
     exactly (IEEE subtraction is antisymmetric)."""
