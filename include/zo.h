@@ -150,6 +150,26 @@ ZO_API int zo_probe_losses_slice(zo_ctx* ctx, const float* theta_dev, uint64_t s
 ZO_API int zo_coeffs(zo_ctx* ctx, const float* loss_plus_dev, const float* loss_minus_dev,
               int32_t n_pert, float eps, float eta, float* coeffs_dev, void* stream);
 
+/* L(theta): the mean cross-entropy of the unperturbed forward over the scored
+ * targets of tokens_dev / targets_dev (int32 [batch x seq], device), written
+ * to loss_dev (one fp32, device).  It runs the probe-loss path for one probe
+ * at radius 0, so both of its signs are exactly L(theta); the baseline that a
+ * forward difference subtracts, and an exact evaluation loss.  Argument
+ * checks and device errors as zo_probe_losses.  Async. */
+ZO_API int zo_loss(zo_ctx* ctx, const float* theta_dev, const int32_t* tokens_dev,
+                   const int32_t* targets_dev, int32_t batch, int32_t seq, float* loss_dev,
+                   void* stream);
+
+/* Forward-difference coefficients c_i = eta (L+_i - L0) / (eps n_pert), with
+ * L0 = L(theta) from zo_loss (one fp32, device): the one-sided estimator
+ * g_hat = 1/n sum_i (L(theta + eps p_i) - L(theta)) / eps p_i, applied by
+ * zo_update like the central coefficients.  Over an antithetic probe set
+ * {p_i, -p_i} it equals the central difference (review, "Circularity Check":
+ * Appendix C).  Non-finite inputs as in zo_coeffs.  Async. */
+ZO_API int zo_coeffs_forward(zo_ctx* ctx, const float* loss_plus_dev, const float* loss0_dev,
+                             int32_t n_pert, float eps, float eta, float* coeffs_dev,
+                             void* stream);
+
 /* theta_j -= sum_i c_i p_ij for every real parameter j, probes replayed from
  * (step_seed, i) and never stored (review, "What carries the argument").
  * theta_dev is updated in place; padding stays zero.  For ZO_DTYPE_BF16 the

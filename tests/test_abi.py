@@ -68,6 +68,9 @@ def test_argument_errors_need_no_device(lib):
     assert lib.zo_probe_losses(None, None, 0, 1, 1e-3, None, None, 1, 1, None, None, None) == \
         zo.ZO_ERR_INVALID_ARG
     assert lib.zo_update(None, None, 0, 1, None, None) == zo.ZO_ERR_INVALID_ARG
+    assert lib.zo_loss(None, None, None, None, 1, 1, None, None) == zo.ZO_ERR_INVALID_ARG
+    assert lib.zo_coeffs_forward(None, None, None, 1, 1e-3, 1e-3, None, None) == \
+        zo.ZO_ERR_INVALID_ARG
     assert lib.zo_sign_words(0, -1, 0, 1, None, None) == zo.ZO_ERR_INVALID_ARG
 
 

@@ -109,6 +109,45 @@ def test_update_matches_oracle(name, n):
         _check_update(cfg, n, theta, seed, coeffs, ctx)
 
 
+@pytest.mark.parametrize("kind", ["tiny", "overfit", "bf16", "bf16_vocab"])
+def test_unperturbed_loss_matches_oracle(kind):
+    """zo_loss: the forward at radius 0 on every forward path (per-probe fp32,
+    probe-column fp32, bf16 tensor cores, bf16 with the vocabulary table)."""
+    if kind in ("tiny", "overfit"):
+        cfg = W.CONFIGS[kind]
+        theta = W.init_theta(cfg)
+        tok, tgt = W.batch_for(cfg)
+        ctx = zo.Context.for_config(cfg)
+        rtol = 1e-5
+    else:
+        E = 64 if kind == "bf16" else 512
+        cfg = W.small_config(vocab=50, embed=E, hidden=64, layers=2, dtype="bf16")
+        theta = W.init_theta(cfg, seed=4)
+        tok, tgt = W.random_batch(256, 3, 50, seed=6, ignore_frac=0.2)
+        ctx = zo.Context(50, E, 64, 2, "bf16", 256, 3, 0)
+        rtol = 1e-2
+    spec = (cfg.vocab, cfg.embed, cfg.hidden, cfg.layers)
+    with ctx:
+        out = torch.full((1,), float("nan"), device="cuda")
+        zo.zo_loss(ctx, dev(theta), dev(tok), dev(tgt), out)
+        assert zo.zo_sync_status(ctx) == zo.ZO_OK
+        got = float(out.cpu())
+    assert math.isclose(got, O.loss_at(theta, spec, tok, tgt), rel_tol=rtol)
+
+
+def test_forward_coefficients_match_formula():
+    n = 257
+    rng = np.random.default_rng(4)
+    lp = (2.3 + 1e-3 * rng.standard_normal(n)).astype(np.float32)
+    l0 = np.float32(2.3)
+    with zo.Context(10, 16, 32, 1) as ctx:
+        out = torch.empty(n, device="cuda")
+        zo.zo_coeffs_forward(ctx, dev(lp), dev(np.array([l0])), n, 1e-3, 5e-2, out)
+        assert zo.zo_sync_status(ctx) == zo.ZO_OK
+        want = O.coefficients_forward(lp, float(l0), n, 1e-3, 5e-2)
+        assert np.allclose(out.cpu().numpy(), want, rtol=1e-6, atol=0)
+
+
 def test_update_rejects_too_many_probes():
     cfg = W.CONFIGS["tiny"]
     n = zo.ZO_MAX_UPDATE_PROBES + 1

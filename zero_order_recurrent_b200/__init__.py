@@ -32,7 +32,7 @@ EXPORTS = (
     "zo_probe_losses_ex", "zo_coeffs", "zo_update", "zo_invalidate_shadow", "zo_step_host",
     "zo_sync_status", "zo_sign_words", "zo_status_string", "zo_kernel_launches",
     "zo_debug_cell_preact", "zo_profile", "zo_profile_read", "zo_probe_losses_static",
-    "zo_probe_losses_slice",
+    "zo_probe_losses_slice", "zo_loss", "zo_coeffs_forward",
 )
 ZO_STATIC_SCRATCH_FLOATS = 65536
 ZO_MAX_UPDATE_PROBES = 8192
@@ -73,6 +73,8 @@ def load_library(path: str = LIB_PATH):
         "zo_probe_losses_ex": ([P, P, U64, I32, F, P, P, I32, I32, P, P, P, P], ctypes.c_int),
         "zo_coeffs": ([P, P, P, I32, F, F, P, P], ctypes.c_int),
         "zo_update": ([P, P, U64, I32, P, P], ctypes.c_int),
+        "zo_loss": ([P, P, P, P, I32, I32, P, P], ctypes.c_int),
+        "zo_coeffs_forward": ([P, P, P, I32, F, F, P, P], ctypes.c_int),
         "zo_invalidate_shadow": ([P], ctypes.c_int),
         "zo_step_host": ([P, P, U64, I32, F, F, P, P, I32, I32, P, P, P], ctypes.c_int),
         "zo_sync_status": ([P, P], ctypes.c_int),
@@ -196,6 +198,19 @@ def zo_probe_losses_slice(ctx, theta, step_seed, probe_begin, n_probes, eps, tok
 def zo_coeffs(ctx, loss_plus, loss_minus, n_pert, eps, eta, coeffs, stream=None):
     _check(load_library().zo_coeffs(ctx.handle, _ptr(loss_plus), _ptr(loss_minus), n_pert, eps,
                                     eta, _ptr(coeffs), _stream(stream)), "zo_coeffs")
+
+
+def zo_loss(ctx, theta, tokens, targets, loss, stream=None):
+    """L(theta) of the unperturbed forward into `loss` (one float, device)."""
+    B, T = tokens.shape
+    _check(load_library().zo_loss(ctx.handle, _ptr(theta), _ptr(tokens), _ptr(targets), B, T,
+                                  _ptr(loss), _stream(stream)), "zo_loss")
+
+
+def zo_coeffs_forward(ctx, loss_plus, loss0, n_pert, eps, eta, coeffs, stream=None):
+    _check(load_library().zo_coeffs_forward(ctx.handle, _ptr(loss_plus), _ptr(loss0), n_pert, eps,
+                                            eta, _ptr(coeffs), _stream(stream)),
+           "zo_coeffs_forward")
 
 
 def zo_update(ctx, theta, step_seed, n_pert, coeffs, stream=None):

@@ -85,6 +85,30 @@ cudaError_t launch_coeffs(const float* lp, const float* lm, int n, float eps, fl
   return cudaGetLastError();
 }
 
+// Forward-difference coefficients c_i = eta (L+_i - L0) / (eps n_pert).
+__global__ void coeffs_forward_kernel(const float* lp, const float* l0, int n, float eps,
+                                      float eta, float* out, unsigned* err) {
+  const float scale = eta / (eps * (float)n);
+  const float b = *l0;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+    const float a = lp[i];
+    float c = (a - b) * scale;
+    if (!isfinite(a) || !isfinite(b) || !isfinite(c)) {
+      latch(err, kErrNonfinite);
+      c = __int_as_float(0x7fc00000);
+    }
+    out[i] = c;
+  }
+}
+
+cudaError_t launch_coeffs_forward(const float* lp, const float* l0, int n, float eps, float eta,
+                                  float* out, unsigned* err, cudaStream_t st) {
+  const int grid = (n + 255) / 256;
+  coeffs_forward_kernel<<<grid, 256, 0, st>>>(lp, l0, n, eps, eta, out, err);
+  count_launch();
+  return cudaGetLastError();
+}
+
 // ---------------------------------------------------------------------------
 // Update.  theta'_j = theta_j + sum_i (-c_i) p_ij is evaluated four probes at
 // a time through subset-sum tables: for the probes 4g..4g+3 of group g,

@@ -102,6 +102,7 @@ void free_ctx(zo_ctx* c) {
   cudaFree(c->coef);
   cudaFree(c->wt);
   cudaFree(c->vt);
+  cudaFree(c->l0m);
   for (auto& r : c->prof) {
     if (r.a) cudaEventDestroy(r.a);
     if (r.b) cudaEventDestroy(r.b);
@@ -177,6 +178,7 @@ int zo_create(const zo_model_spec* spec, zo_ctx** out) {
   };
   alloc((void**)&c->err, sizeof(unsigned));
   if (rc == ZO_OK) cudaMemset(c->err, 0, sizeof(unsigned));
+  alloc((void**)&c->l0m, sizeof(float));
   alloc((void**)&c->tok, sizeof(int32_t) * B * s.max_seq);
   alloc((void**)&c->tgt, sizeof(int32_t) * B * s.max_seq);
 
@@ -291,13 +293,15 @@ int zo_invalidate_shadow(zo_ctx* ctx) {
 // Losses of probes probe_begin .. probe_begin + n_pert - 1 (the probes' signs
 // use their global index), written to loss_plus[i], loss_minus[i] for
 // i < n_pert.
+// radius0: the unperturbed forward (zo_loss), eps must be 0.
 static int probe_losses_range(zo_ctx* ctx, const float* theta, uint64_t seed, int32_t probe_begin,
                               int32_t n_pert, float eps, const int32_t* tokens,
                               const int32_t* targets, int32_t batch, int32_t seq, float* loss_plus,
-                              float* loss_minus, float* row_loss, void* stream) {
+                              float* loss_minus, float* row_loss, void* stream,
+                              bool radius0 = false) {
   if (!ctx || !theta || !tokens || !targets || !loss_plus || !loss_minus) return ZO_ERR_INVALID_ARG;
   if (n_pert < 1 || probe_begin < 0 || (int64_t)probe_begin + n_pert > INT32_MAX ||
-      !(eps > 0.f) || !isfinite(eps))
+      !(radius0 ? eps == 0.f : (eps > 0.f && isfinite(eps))))
     return ZO_ERR_INVALID_ARG;
   if (batch < 1 || batch > ctx->spec.max_batch || seq < 1 || seq > ctx->spec.max_seq)
     return ZO_ERR_INVALID_ARG;
@@ -402,6 +406,23 @@ int zo_coeffs(zo_ctx* ctx, const float* lp, const float* lm, int32_t n, float ep
   if (!(eps > 0.f) || !isfinite(eps) || !isfinite(eta)) return ZO_ERR_INVALID_ARG;
   ZO_CUDA(timed(ctx, S(stream), ZO_KIND_OTHER, 0.0, 0.0, [&] {
     return launch_coeffs(lp, lm, n, eps, eta, coeffs, ctx->err, S(stream));
+  }));
+  return ZO_OK;
+}
+
+int zo_loss(zo_ctx* ctx, const float* theta, const int32_t* tokens, const int32_t* targets,
+            int32_t batch, int32_t seq, float* loss, void* stream) {
+  if (!ctx || !loss) return ZO_ERR_INVALID_ARG;
+  return probe_losses_range(ctx, theta, 0, 0, 1, 0.f, tokens, targets, batch, seq, loss, ctx->l0m,
+                            nullptr, stream, true);
+}
+
+int zo_coeffs_forward(zo_ctx* ctx, const float* lp, const float* l0, int32_t n, float eps,
+                      float eta, float* coeffs, void* stream) {
+  if (!ctx || !lp || !l0 || !coeffs || n < 1) return ZO_ERR_INVALID_ARG;
+  if (!(eps > 0.f) || !isfinite(eps) || !isfinite(eta)) return ZO_ERR_INVALID_ARG;
+  ZO_CUDA(timed(ctx, S(stream), ZO_KIND_OTHER, 0.0, 0.0, [&] {
+    return launch_coeffs_forward(lp, l0, n, eps, eta, coeffs, ctx->err, S(stream));
   }));
   return ZO_OK;
 }

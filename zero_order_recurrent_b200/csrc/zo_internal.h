@@ -79,6 +79,7 @@ struct zo_ctx {
   float* lm = nullptr;
   float* coef = nullptr;
   int n_stage = 0;               // capacity of lp/lm/coef
+  float* l0m = nullptr;          // zo_loss: the second sign's copy of L(theta)
   int fp32_bb = 1;               // rows per CTA of the fp32 forward
   size_t fp32_smem = 0;
   int fp32_wide_np = 0;          // probes per CTA of the probe-column fp32 forward (0: unused)
@@ -101,6 +102,8 @@ cudaError_t launch_cast_shadow(const float* theta, __nv_bfloat16* shadow, int64_
                                cudaStream_t st);
 cudaError_t launch_coeffs(const float* lp, const float* lm, int n, float eps, float eta,
                           float* out, unsigned* err, cudaStream_t st);
+cudaError_t launch_coeffs_forward(const float* lp, const float* l0, int n, float eps, float eta,
+                                  float* out, unsigned* err, cudaStream_t st);
 cudaError_t launch_update(const zo_ctx* ctx, float* theta, uint64_t seed, int n,
                           const float* coeffs, __nv_bfloat16* shadow, cudaStream_t st);
 cudaError_t launch_fp32_forward(const zo_ctx* ctx, const float* theta, uint64_t seed, int probe0,

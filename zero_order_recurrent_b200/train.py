@@ -8,8 +8,8 @@ This driver runs that loop on one GPU: every step draws a fresh batch of
 lengths 1..max_len, calls zo_probe_losses / zo_coeffs / zo_update (the
 probes are replayed from the step seed, never stored), and records the loss
 at theta estimated as the mean of (L+ + L-)/2 over the probes (O(eps^2) from
-L(theta)).  After training, each evaluation length is scored the same way with
-one probe.
+L(theta)).  After training, each evaluation length is scored by zo_loss, the
+unperturbed forward.
 
     python -m zero_order_recurrent_b200.train --task copy --steps 2000 --eta 0.05
 """
@@ -30,9 +30,13 @@ def _repo_root():
 def train(task: str = "copy", steps: int = 1000, n_pert: int = 64, eps: float = 1e-3,
           eta: float = 1e-3, batch: int = 8, max_len: int = 10, eval_lengths=(11, 20, 40, 60),
           embed: int = 16, hidden: int = 32, layers: int = 1, seed: int = 0,
-          log_every: int = 100, theta=None):
-    """Runs `steps` CD-RGE updates; returns the loss history, the evaluation
-    losses per length, the device time per step and the final theta (device)."""
+          log_every: int = 100, theta=None, estimator: str = "central"):
+    """Runs `steps` zero-order updates; returns the loss history, the evaluation
+    losses per length, the device time per step and the final theta (device).
+    estimator "central": c_i = eta (L+_i - L-_i)/(2 eps n) (CD-RGE);
+    "forward": c_i = eta (L+_i - L(theta))/(eps n) with L(theta) from zo_loss."""
+    if estimator not in ("central", "forward"):
+        raise ValueError(f"unknown estimator {estimator}")
     import torch
     if _repo_root() not in sys.path:
         sys.path.insert(0, _repo_root())
@@ -49,6 +53,7 @@ def train(task: str = "copy", steps: int = 1000, n_pert: int = 64, eps: float = 
     lp = torch.empty(n_pert, device=dev)
     lm = torch.empty(n_pert, device=dev)
     coef = torch.empty(n_pert, device=dev)
+    l0 = torch.empty(1, device=dev)
     rng = np.random.default_rng(seed)
     history = []
     ms = 0.0
@@ -61,8 +66,14 @@ def train(task: str = "copy", steps: int = 1000, n_pert: int = 64, eps: float = 
             e0 = torch.cuda.Event(enable_timing=True)
             e1 = torch.cuda.Event(enable_timing=True)
             e0.record()
-            zo.cdrge_step(ctx, theta, W.step_seed(step, run_seed=seed), n_pert, eps, eta, tok_d,
-                          tgt_d, lp, lm, coef)
+            sseed = W.step_seed(step, run_seed=seed)
+            if estimator == "central":
+                zo.cdrge_step(ctx, theta, sseed, n_pert, eps, eta, tok_d, tgt_d, lp, lm, coef)
+            else:
+                zo.zo_loss(ctx, theta, tok_d, tgt_d, l0)
+                zo.zo_probe_losses(ctx, theta, sseed, n_pert, eps, tok_d, tgt_d, lp, lm)
+                zo.zo_coeffs_forward(ctx, lp, l0, n_pert, eps, eta, coef)
+                zo.zo_update(ctx, theta, sseed, n_pert, coef)
             e1.record()
             if step % log_every == 0 or step == steps - 1:
                 torch.cuda.synchronize()
@@ -76,15 +87,15 @@ def train(task: str = "copy", steps: int = 1000, n_pert: int = 64, eps: float = 
         for L in eval_lengths:
             tok, tgt = W.transduction_batch(task, [L] * batch, W.task_length(task, L),
                                             seed=seed * 1000003 + 10**9 + L)
-            zo.zo_probe_losses(ctx, theta, W.step_seed(10**6 + L, run_seed=seed), 1, eps,
-                               torch.from_numpy(tok).to(dev), torch.from_numpy(tgt).to(dev),
-                               lp[:1], lm[:1])
+            zo.zo_loss(ctx, theta, torch.from_numpy(tok).to(dev), torch.from_numpy(tgt).to(dev),
+                       lp[:1])
             torch.cuda.synchronize()
-            evals[int(L)] = float((lp[0] + lm[0]) * 0.5)
+            evals[int(L)] = float(lp[0])
         st = zo.zo_sync_status(ctx)
         if st != zo.ZO_OK:
             raise RuntimeError(f"evaluation: {zo.status_string(st)}")
-    return {"task": task, "steps": steps, "n_pert": n_pert, "eps": eps, "eta": eta,
+    return {"task": task, "estimator": estimator, "steps": steps, "n_pert": n_pert, "eps": eps,
+            "eta": eta,
             "max_len": max_len, "history": history, "eval": evals,
             "ms_per_step": ms / max(steps, 1), "theta": theta}
 
@@ -103,11 +114,13 @@ def main(argv=None):
     ap.add_argument("--hidden", type=int, default=32)
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--log-every", type=int, default=100)
+    ap.add_argument("--estimator", default="central", choices=["central", "forward"])
     args = ap.parse_args(argv)
     for eta in args.eta:
         r = train(task=args.task, steps=args.steps, n_pert=args.n_pert, eps=args.eps, eta=eta,
                   batch=args.batch, max_len=args.max_len, eval_lengths=args.eval_lengths,
-                  hidden=args.hidden, seed=args.seed, log_every=args.log_every)
+                  hidden=args.hidden, seed=args.seed, log_every=args.log_every,
+                  estimator=args.estimator)
         r.pop("theta")
         print(json.dumps(r), flush=True)
 
