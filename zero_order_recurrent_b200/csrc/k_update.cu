@@ -1,7 +1,7 @@
-// Coefficients and the seed-replayed update (pith.science review, "What
-// carries the argument": Theta' = Theta - 1/(2 n_pert) sum_i (L+_i - L-_i) p_i;
-// alex-wiki "Method": theta' = theta - eta g_hat), plus the probe-sign test
-// hook and the bf16 shadow cast.
+// Coefficients (central and forward-difference) and the seed-replayed update
+// (pith.science review, "What carries the argument": Theta' = Theta -
+// 1/(2 n_pert) sum_i (L+_i - L-_i) p_i; alex-wiki "Method": theta' = theta -
+// eta g_hat), plus the probe-sign test hook and the bf16 shadow cast.
 #include "zo_common.cuh"
 #include "zo_internal.h"
 
