@@ -257,7 +257,8 @@ struct TcCfg {
   static constexpr int STAGE = A_BYTES + B_BYTES;
   static constexpr int COLS = MT * BN;              // TMEM columns per accumulator
   static constexpr int TMEM_COLS = COLS * ACC;
-  static constexpr int SMEM = STAGES * STAGE + 1024 + 256;
+  static constexpr int EPI = 4 * 4 * U * 4;          // per epilogue warp: bias slice [4][U]
+  static constexpr int SMEM = STAGES * STAGE + 1024 + 256 + EPI;
   static_assert(BN % 64 == 0 && BN <= 256, "BN");
   static_assert(TMEM_COLS == 128 || TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM columns");
 };
@@ -480,12 +481,25 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // ------------------------------------------------------------ epilogue
     const int quad = warp & 3;
     const int rloc = quad * 32 + lane;
+    // this warp's copy of the tile's bias slice [4 gates][U units]
+    float* bias_s = reinterpret_cast<float*>(smem + STAGES * C::STAGE + 256) + quad * 4 * C::U;
     uint32_t tcount = 0;
     bool ok = true;
     for (int64_t tile = blockIdx.x; tile < a.tiles && ok; tile += gridDim.x, ++tcount) {
       const TileCoord tc = decode_tile(a, tile, P);
       const int ab = tcount % ACC;
       const uint32_t aph = (tcount / ACC) & 1;
+      if constexpr (MODE == 0 || MODE == 2) {
+        // staged while the tile's MMAs run, so the epilogue's bias reads are
+        // shared-memory broadcasts instead of one L2 round trip per chunk
+        const float* bsrc = a.small_p + tc.ps * a.sstride + a.soffb + tc.n * C::U;
+        __syncwarp();
+        for (int i = lane; i < 4 * C::U; i += 32) {
+          const int g = i / C::U;
+          bias_s[i] = __ldg(bsrc + g * a.H + (i - g * C::U));
+        }
+        __syncwarp();
+      }
       if ((MODE == 0 || MODE == 2) && !a.first && !a.raw) {
         // while this tile's MMAs run, pull its c_{t-1} rows (and the token's
         // vocabulary-table rows) into L2 so the epilogue's loads hit L2
@@ -554,15 +568,44 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const bool live = b < a.B;
         const bool need_c = live && !a.first && !a.raw;
         float4* crow = reinterpret_cast<float4*>(a.cst + rowoff + tc.n * C::U);
-        // c_{t-1} of the next 8-unit chunk is loaded one chunk ahead, so its
-        // latency overlaps this chunk's TMEM load and gate arithmetic
-        float4 cn0 = make_float4(0.f, 0.f, 0.f, 0.f), cn1 = cn0;
+        // input term from the vocabulary table: the row of this batch row's token
+        const float* trow = nullptr;
+        if constexpr (MODE == 2) {
+          if (live) {
+            int tok = a.tokens[(int64_t)b * a.T + a.t];
+            if (tok < 0 || tok >= a.V) {
+              latch(a.err, kErrBounds);
+              tok = 0;
+            }
+            trow = a.vt + ((int64_t)tc.ps * a.vtrows + tok) * 4 * a.H + tc.n * C::U;
+          }
+        }
+        // c_{t-1} is loaded two 8-unit chunks ahead (one with the table, whose
+        // loads need the registers), so its latency overlaps the TMEM loads
+        // and gate arithmetic of the chunks before
+        constexpr bool kTwoAhead = MODE != 2;
+        float4 cn0 = make_float4(0.f, 0.f, 0.f, 0.f), cn1 = cn0, cm0 = cn0, cm1 = cn0;
         if (need_c) {
           cn0 = crow[0];
           cn1 = crow[1];
+          if (kTwoAhead && 8 < C::U) {
+            cm0 = crow[2];
+            cm1 = crow[3];
+          }
         }
 #pragma unroll 1
         for (int u0 = 0; u0 < C::U; u0 += 8) {
+          // table loads issued before the TMEM loads: their latency overlaps the wait
+          float4 tv[4][2];
+          if constexpr (MODE == 2) {
+            if (live) {
+#pragma unroll
+              for (int g = 0; g < 4; ++g)
+#pragma unroll
+                for (int q4 = 0; q4 < 2; ++q4)
+                  tv[g][q4] = __ldg(reinterpret_cast<const float4*>(trow + g * a.H + u0) + q4);
+            }
+          }
           uint32_t acc[4][8];
 #pragma unroll
           for (int g = 0; g < 4; ++g)
@@ -570,7 +613,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                          g * C::U + u0,
                      acc[g]);
           const float4 cc0 = cn0, cc1 = cn1;
-          if (need_c && u0 + 8 < C::U) {
+          if constexpr (kTwoAhead) {
+            cn0 = cm0;
+            cn1 = cm1;
+            if (need_c && u0 + 16 < C::U) {
+              cm0 = crow[(u0 >> 2) + 4];
+              cm1 = crow[(u0 >> 2) + 5];
+            }
+          } else if (need_c && u0 + 8 < C::U) {
             cn0 = crow[(u0 >> 2) + 2];
             cn1 = crow[(u0 >> 2) + 3];
           }
@@ -578,28 +628,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           if (live) {
             const int unit0 = tc.n * C::U + u0;
             float pre[4][8];
-            // input term from the vocabulary table (row of this batch row's token)
-            const float* trow = nullptr;
-            if constexpr (MODE == 2) {
-              int tok = a.tokens[(int64_t)b * a.T + a.t];
-              if (tok < 0 || tok >= a.V) {
-                latch(a.err, kErrBounds);
-                tok = 0;
-              }
-              trow = a.vt + ((int64_t)tc.ps * a.vtrows + tok) * 4 * a.H + unit0;
-            }
 #pragma unroll
             for (int g = 0; g < 4; ++g) {
-              const float4* bp = reinterpret_cast<const float4*>(bias + g * a.H + unit0);
+              const float4* bp = reinterpret_cast<const float4*>(bias_s + g * C::U + u0);
 #pragma unroll
               for (int q4 = 0; q4 < 2; ++q4) {
-                float4 bv = MODE == 3 ? make_float4(0.f, 0.f, 0.f, 0.f) : __ldg(bp + q4);
+                float4 bv = MODE == 3 ? make_float4(0.f, 0.f, 0.f, 0.f) : bp[q4];
                 if constexpr (MODE == 2) {
-                  const float4 tv = __ldg(reinterpret_cast<const float4*>(trow + g * a.H) + q4);
-                  bv.x += tv.x;
-                  bv.y += tv.y;
-                  bv.z += tv.z;
-                  bv.w += tv.w;
+                  bv.x += tv[g][q4].x;
+                  bv.y += tv[g][q4].y;
+                  bv.z += tv[g][q4].z;
+                  bv.w += tv[g][q4].w;
                 }
                 pre[g][4 * q4 + 0] = __uint_as_float(acc[g][4 * q4 + 0]) + bv.x;
                 pre[g][4 * q4 + 1] = __uint_as_float(acc[g][4 * q4 + 1]) + bv.y;
