@@ -26,6 +26,13 @@ MUTATIONS = {
     "philox_swapped_multipliers": ("p0 = c0 * np.uint64(PHILOX_M0)", "p0 = c0 * np.uint64(PHILOX_M1)"),
     "lse_without_max": ("lse = m[:, 0] + np.log", "lse = np.log"),
     "perturb_ignores_sign": ("+ sign * e * p", "+ e * p"),
+    "gram_cosine_no_sqrt": ("den = math.sqrt(max(a @ gram @ a, 0.0) * max(b @ gram @ b, 0.0))",
+                            "den = max(a @ gram @ a, 0.0) * max(b @ gram @ b, 0.0)"),
+    "gram_cosine_ignores_gram": ("num = a @ gram @ b", "num = a @ b"),
+    "gram_counts_padding": ("        cnt = r * c\n        S = np.stack",
+                            "        cnt = -(-(r * c) // 128) * 128\n        S = np.stack"),
+    "gram_ignores_probe_list": ("S = np.stack([probe_signs(step_seed, i, off, cnt).astype(np.int64) for i in probes])",
+                                "S = np.stack([probe_signs(step_seed, i, off, cnt).astype(np.int64) for i in range(n)])"),
 }
 
 
@@ -44,6 +51,9 @@ PIN_FUNCS = [
     pins.test_quadratic_all_sign_vectors_give_exact_gradient,
     pins.test_central_difference_matches_directional_derivative,
     pins.test_antisymmetry_negated_probe_negates_coefficient,
+    pins.test_probe_gram_matches_explicit_products,
+    pins.test_gram_cosine_hand_values,
+    pins.test_gram_cosine_equals_cosine_of_explicit_estimates,
 ]
 
 

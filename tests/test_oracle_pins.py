@@ -392,3 +392,55 @@ def test_update_replays_probes():
     assert np.array_equal(new[~mask], theta[~mask].astype(np.float64))
     idx = np.nonzero(mask)[0][::37]
     assert np.allclose(O.update_at(theta, seed, cfg.n_pert, c, idx), new[idx], rtol=0, atol=1e-15)
+
+
+# ---------------------------------------------------------------------------
+# The cosine gate of the GPU tests: probe Gram matrix and cos(g_a, g_b)
+# ---------------------------------------------------------------------------
+def test_probe_gram_matches_explicit_products():
+    """probe_gram (per-segment sign products over the real parameters) equals
+    P P^T of the explicit probe matrix (padding columns 0) for a subset of
+    probes in any order; its diagonal is d_real (closed form)."""
+    cfg = W.small_config(vocab=5, embed=3, hidden=7, layers=2)
+    spec = (cfg.vocab, cfg.embed, cfg.hidden, cfg.layers)
+    seed = W.step_seed(8)
+    P = O.probe_matrix(spec, seed, 6).astype(np.int64)
+    sel = [4, 1, 5]
+    G = O.probe_gram(spec, seed, sel)
+    assert np.array_equal(G, (P @ P.T)[np.ix_(sel, sel)])
+    d_real = cfg.vocab * cfg.embed + sum(4 * cfg.hidden * ((cfg.embed if l == 0 else cfg.hidden)
+                                                           + cfg.hidden) + 4 * cfg.hidden
+                                         for l in range(cfg.layers)) + cfg.vocab * cfg.hidden + cfg.vocab
+    assert np.all(np.diag(G) == d_real)
+
+
+def test_gram_cosine_hand_values():
+    """cos(sum a_i p_i, sum b_i p_i) from the Gram matrix.  Orthonormal probes
+    (G = I): orthogonal coefficients give 0, proportional 1, opposite -1,
+    (3, 4) vs (4, 3) gives 24/25.  Probes (1,1,1) and (1,1,-1) (G = [[3,1],[1,3]]):
+    the two probes themselves have cosine 1/3."""
+    I = np.eye(2)
+    assert O.gram_cosine([1, 0], [0, 1], I) == 0.0
+    assert math.isclose(O.gram_cosine([1, 2], [2, 4], I), 1.0, rel_tol=1e-15)
+    assert math.isclose(O.gram_cosine([1, 2], [-1, -2], I), -1.0, rel_tol=1e-15)
+    assert math.isclose(O.gram_cosine([3, 4], [4, 3], I), 24 / 25, rel_tol=1e-15)
+    G = np.array([[3.0, 1.0], [1.0, 3.0]])
+    assert math.isclose(O.gram_cosine([1, 0], [0, 1], G), 1 / 3, rel_tol=1e-15)
+    assert math.isclose(O.gram_cosine([2, 0], [0, 5], G), 1 / 3, rel_tol=1e-15)
+
+
+def test_gram_cosine_equals_cosine_of_explicit_estimates():
+    """On Philox probes, gram_cosine(a, b, probe_gram) is the plain cosine of the
+    explicit vectors sum a_i p_i and sum b_i p_i built from the probe matrix."""
+    cfg = W.CONFIGS["tiny"]
+    spec = (cfg.vocab, cfg.embed, cfg.hidden, cfg.layers)
+    seed = W.step_seed(5)
+    n = 6
+    rng = np.random.default_rng(2)
+    a = rng.standard_normal(n)
+    b = a + 0.3 * rng.standard_normal(n)
+    P = O.probe_matrix(spec, seed, n).astype(np.float64)
+    ga, gb = a @ P, b @ P
+    want = float(ga @ gb / (np.linalg.norm(ga) * np.linalg.norm(gb)))
+    got = O.gram_cosine(a, b, O.probe_gram(spec, seed, range(n)))
+    assert math.isclose(got, want, rel_tol=1e-12)
