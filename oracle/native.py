@@ -54,6 +54,7 @@ def _declare(lib):
         "zoo_coefficients": ([P, P, I32, F, F, P], None),
         "zoo_coefficients_forward": ([P, D, I32, F, F, P], None),
         "zoo_update": ([P, I32, I32, I32, I32, U64, I32, P, P, I64, I32, P], I32),
+        "zoo_update_range": ([P, I32, I32, I32, I32, U64, I32, P, I64, I64, I32, P], I32),
         "zoo_probe_gram": ([I32, I32, I32, I32, U64, P, I32, I32, P], I32),
     }
     for name, (args, res) in sig.items():
@@ -171,6 +172,17 @@ class Oracle:
         out = np.zeros(th.size)
         if self.lib.zoo_update(_p(th), V, E, H, L, step_seed, n_pert, _p(c), None, 0,
                                threads or cores(), _p(out)):
+            raise ValueError("bad arguments to the C++ oracle")
+        return out
+
+    def update_range(self, theta, spec, step_seed, n_pert, coeffs, j0, j1, threads=None):
+        """theta' on the contiguous elements j0 <= j < j1."""
+        V, E, H, L = spec
+        th = self._theta(theta, spec)
+        c = np.ascontiguousarray(coeffs, dtype=np.float64)
+        out = np.zeros(max(j1 - j0, 0))
+        if self.lib.zoo_update_range(_p(th), V, E, H, L, step_seed, n_pert, _p(c), j0, j1,
+                                     threads or cores(), _p(out)):
             raise ValueError("bad arguments to the C++ oracle")
         return out
 

@@ -386,6 +386,9 @@ void zoo_coefficients_forward(const double* lp, double l0, int n, float eps, flo
   for (int i = 0; i < n; ++i) out[i] = (double)eta * (lp[i] - l0) / ((double)eps * n);
 }
 
+int zoo_update_range(const float* theta, int V, int E, int H, int L, uint64_t seed, int n_pert,
+                     const double* coeffs, int64_t j0, int64_t j1, int threads, double* out);
+
 // theta'_j = theta_j - sum_i c_i p_ij for the elements index[0..n_index), or
 // for all d_pad elements when index is null (padding copied unchanged).
 // out: fp64 [n_index] or [d_pad].  Returns 1 on bad arguments.
@@ -410,9 +413,23 @@ int zoo_update(const float* theta, int V, int E, int H, int L, uint64_t seed, in
     });
     return 0;
   }
-  for (int64_t j = 0; j < m.d_pad; ++j) out[j] = (double)theta[j];
+  return zoo_update_range(theta, V, E, H, L, seed, n_pert, coeffs, 0, m.d_pad, threads, out);
+}
+
+// theta'_j for the contiguous elements j0 <= j < j1 (out: fp64 [j1 - j0];
+// padding copied unchanged).  Returns 1 on bad arguments.
+int zoo_update_range(const float* theta, int V, int E, int H, int L, uint64_t seed, int n_pert,
+                     const double* coeffs, int64_t j0_all, int64_t j1_all, int threads,
+                     double* out) {
+  const Layout m = make_layout(V, E, H, L);
+  if (!theta || !coeffs || !out || n_pert < 0 || threads < 1 || j0_all < 0 || j1_all > m.d_pad ||
+      j0_all > j1_all)
+    return 1;
+  for (int64_t j = j0_all; j < j1_all; ++j) out[j - j0_all] = (double)theta[j];
   for (size_t s = 0; s < m.seg_off.size(); ++s) {
-    const int64_t off = m.seg_off[s], len = m.seg_len[s];
+    const int64_t off = std::max(m.seg_off[s], j0_all);
+    const int64_t len = std::min(m.seg_off[s] + m.seg_len[s], j1_all) - off;
+    if (len <= 0) continue;
     const int64_t nblk = (len + 4095) / 4096;
     parallel_for(nblk, nblk >= 4 ? threads : 1, [&](int64_t b0, int64_t b1) {
       std::vector<double> p(4096);
@@ -421,7 +438,7 @@ int zoo_update(const float* theta, int V, int E, int H, int L, uint64_t seed, in
         const int64_t n = std::min<int64_t>(4096, off + len - j0);
         for (int i = 0; i < n_pert; ++i) {
           signs(seed, (uint32_t)i, j0, n, p.data());
-          for (int64_t k = 0; k < n; ++k) out[j0 + k] -= coeffs[i] * p[k];
+          for (int64_t k = 0; k < n; ++k) out[j0 - j0_all + k] -= coeffs[i] * p[k];
         }
       }
     });

@@ -122,6 +122,8 @@ def pin_update_matches_explicit_sum(N):
     assert np.array_equal(new[~mask], theta[~mask].astype(np.float64))
     idx = np.nonzero(mask)[0][::11]
     assert np.allclose(N.update_at(theta, spec, seed, n, c, idx), new[idx], rtol=0, atol=1e-15)
+    for j0, j1 in ((0, len(theta)), (5, 300), (200, 201), (130, 130)):
+        assert np.array_equal(N.update_range(theta, spec, seed, n, c, j0, j1, threads=2), new[j0:j1])
 
 
 def pin_gram_matches_explicit(N):
@@ -216,7 +218,8 @@ MUTATIONS = {
     "philox_swapped_multipliers": ("(uint64_t)0xD2511F53u * x[0]", "(uint64_t)0xCD9E8D57u * x[0]"),
     "plain_bit_order": ("return (e >> 1) + 16 * (e & 1);", "return e;"),
     "missing_factor_two": ("/ (2.0 * (double)eps * n)", "/ ((double)eps * n)"),
-    "wrong_update_sign": ("out[j0 + k] -= coeffs[i] * p[k];", "out[j0 + k] += coeffs[i] * p[k];"),
+    "wrong_update_sign": ("out[j0 - j0_all + k] -= coeffs[i] * p[k];",
+                          "out[j0 - j0_all + k] += coeffs[i] * p[k];"),
     "perturb_ignores_sign": ("const double step[2] = {s_eps, -s_eps};",
                              "const double step[2] = {s_eps, s_eps};"),
     "lse_without_max": ("row_loss[b] += mx + std::log(se) - zb[tg];",
