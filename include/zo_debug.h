@@ -23,6 +23,22 @@
 extern "C" {
 #endif
 
+/*
+ * zo_debug_cell_stall exercises the bounded device waits (every mbarrier wait
+ * of the tensor-core kernels gives up after a time limit, latches
+ * ZO_ERR_TIMEOUT in the context's error word and returns).  It launches one
+ * tensor-core kernel on the context's own buffers with every wait bounded by
+ * wait_ns and with a producer that issues no copy, so no stage ever fills:
+ *   kind 0  the CTA-pair cell step of layer 0 (tcgen05.mma.cta_group::2);
+ *   kind 1  the single-CTA output layer + cross-entropy (cta_group::1).
+ * All waits run out, the CTAs free their tensor memory and return; no copy and
+ * no MMA is ever in flight, and the context stays usable.  zo_sync_status()
+ * then returns ZO_ERR_TIMEOUT (and clears it).  Only ZO_DTYPE_BF16 contexts
+ * (else ZO_ERR_UNSUPPORTED); wait_ns in [1e3, 1e10] ns (else
+ * ZO_ERR_INVALID_ARG).  Nothing the caller owns is written.  Async on `stream`.
+ */
+ZO_API int zo_debug_cell_stall(zo_ctx* ctx, int32_t kind, uint64_t wait_ns, void* stream);
+
 ZO_API int zo_debug_cell_preact(zo_ctx* ctx, const float* theta_dev, uint64_t step_seed,
                                 int32_t probe0, int32_t n_probes, float eps,
                                 const int32_t* tokens_dev, int32_t batch, int32_t seq,

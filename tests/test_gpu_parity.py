@@ -83,14 +83,21 @@ def _check_update(cfg, n, theta, seed, coeffs, ctx, idx=None):
     c64 = coeffs.astype(np.float32).astype(np.float64)
     if idx is None:
         want = O.update(theta, spec_of(cfg), seed, n, c64)
-        tol = 1e-6 * (np.abs(want) + np.abs(c64).sum())
-        assert np.all(np.abs(got - want) <= tol)
         mask = O.real_mask(*spec_of(cfg))
         assert np.array_equal(got[~mask], theta[~mask])
     else:
         want = O.update_at(theta, seed, n, c64, idx)
-        tol = 1e-6 * (np.abs(want) + np.abs(c64).sum())
-        assert np.all(np.abs(got[idx] - want) <= tol)
+        got = got[idx]
+    err = np.abs(got - want)
+    csum = np.abs(c64).sum()
+    assert np.all(err <= 1e-6 * (np.abs(want) + csum))
+    # where theta' outweighs the coefficient mass, the plain relative bound
+    big = np.abs(want) >= csum
+    if np.any(big):
+        rel = float(np.max(err[big] / np.abs(want[big])))
+        print(f"update n={n}: max relative error {rel:.3e} on {int(big.sum())} elements "
+              f"with |theta'| >= sum|c|")
+        assert rel <= 1e-6
     return th
 
 
@@ -395,51 +402,81 @@ def test_bf16_small_matches_oracle(V, E, H, L, B, T, n):
     assert np.allclose(rows[:, 1], orm, rtol=1e-2, atol=1e-3)
 
 
-def test_bf16_charlm_full_size_two_probes():
-    """charlm exactly as benchmarked (64 probes, batch 1024, T = 10); the oracle
-    evaluates probes 0 and 1 over the whole batch."""
+_NATIVE = None
+
+
+def native_oracle():
+    """The C++ fp64 oracle (built on first use)."""
+    global _NATIVE
+    if _NATIVE is None:
+        from oracle import native
+        _NATIVE = native.Oracle()
+    return _NATIVE
+
+
+def _row_slice_gate(cfg, theta, tok, tgt, seed, rows_gpu, probes, rows):
+    """The GPU's per-row loss sums of a full launch (rows_gpu [n, 2, B]) against
+    the C++ oracle on `probes` x `rows`: every row sum within 1e-2 relative;
+    over the slice, sign(L+ - L-) agreement >= 95% and cos(g_gpu, g_oracle)
+    >= 0.99 (from the probe Gram matrix).  Returns (agreement, cosine)."""
+    NO = native_oracle()
+    spec = spec_of(cfg)
+    orl, orc = NO.probe_row_losses(theta, spec, seed, probes, cfg.eps, tok, tgt, rows=rows)
+    g = rows_gpu[probes][:, :, rows]
+    assert np.allclose(g, orl, rtol=1e-2), float(np.max(np.abs(g - orl) / np.abs(orl)))
+    cnt = orc.sum()
+    glp, glm = g[:, 0].sum(axis=1) / cnt, g[:, 1].sum(axis=1) / cnt
+    olp, olm = orl[:, 0].sum(axis=1) / cnt, orl[:, 1].sum(axis=1) / cnt
+    assert np.allclose(glp, olp, rtol=1e-2) and np.allclose(glm, olm, rtol=1e-2)
+    agree = sign_agreement(glp, glm, olp, olm)
+    cos = O.gram_cosine(glp - glm, olp - olm, NO.probe_gram(spec, seed, probes))
+    print(f"{cfg.name}: {len(probes)} probes x {len(rows)} rows: sign agreement {agree:.4f}, "
+          f"cosine {cos:.5f}")
+    assert agree >= 0.95, agree
+    assert cos >= 0.99, cos
+    return agree, cos
+
+
+def test_bf16_charlm_full_size_all_probes_on_32_rows():
+    """charlm exactly as benchmarked (64 probes, batch 1024, T = 10); the C++
+    oracle evaluates all 64 probes on batch rows 0..31 (each row's forward is
+    independent of the others), compared per row and through the slice's
+    sign agreement and estimate cosine over the 64 probes."""
     cfg = W.CONFIGS["charlm"]
     theta = W.init_theta(cfg)
     tok, tgt = W.batch_for(cfg, step=0)
     seed = W.step_seed(0)
     with zo.Context.for_config(cfg) as ctx:
-        lp, lm = gpu_losses(ctx, theta, seed, cfg.n_pert, cfg.eps, tok, tgt)
-    probes = [0, 1]
-    olp, olm = O.probe_losses(theta, spec_of(cfg), seed, cfg.n_pert, cfg.eps, tok, tgt, probes=probes)
-    assert np.allclose(lp[probes], olp, rtol=1e-2) and np.allclose(lm[probes], olm, rtol=1e-2)
-    assert sign_agreement(lp[probes], lm[probes], olp, olm) >= 0.95
-    assert estimate_cosine(spec_of(cfg), seed, probes, lp[probes], lm[probes], olp, olm) >= 0.99
+        lp, lm, rows = gpu_losses(ctx, theta, seed, cfg.n_pert, cfg.eps, tok, tgt, rows=True)
+    _row_slice_gate(cfg, theta, tok, tgt, seed, rows, list(range(cfg.n_pert)), np.arange(32))
+    n_all = (tgt >= 0).sum()
+    assert np.allclose(lp, rows[:, 0].sum(axis=1) / n_all, rtol=1e-5)
+    assert np.allclose(lm, rows[:, 1].sum(axis=1) / n_all, rtol=1e-5)
 
 
 @pytest.mark.slow
-@pytest.mark.parametrize("name", ["lstm270m", "lstm1b"])
-def test_bf16_large_full_launch_sampled_rows(name):
-    """270M / 1.1B exactly as benchmarked (all probes, batch 1024, T = 10);
-    the oracle evaluates probes 0 and 1 on batch rows 0..31, compared per row
-    (each row's forward is independent of the others), plus the slice losses'
-    sign agreement and the estimate cosine over those probes."""
+@pytest.mark.parametrize("name,n_probes,n_rows", [("lstm270m", 8, 32), ("lstm1b", 2, 32),
+                                                  ("lstm4b", 1, 8)])
+def test_bf16_large_full_launch_sampled_rows(name, n_probes, n_rows):
+    """270M / 1.1B / 4.3B exactly as benchmarked (all probes, batch 1024,
+    T = 10); the C++ oracle evaluates probes 0..n_probes-1 on batch rows
+    0..n_rows-1, compared per row, plus (with two probes or more) the slice's
+    sign agreement and estimate cosine.  The full-batch losses are the means of
+    the GPU's own row sums."""
     cfg = W.CONFIGS[name]
-    spec = spec_of(cfg)
     theta = W.init_theta(cfg)
     tok, tgt = W.batch_for(cfg, step=0)
     seed = W.step_seed(0)
     with zo.Context.for_config(cfg) as ctx:
         lp, lm, rows = gpu_losses(ctx, theta, seed, cfg.n_pert, cfg.eps, tok, tgt, rows=True)
     assert np.all(np.isfinite(lp)) and np.all(np.isfinite(lm))
-    sl = np.arange(32)
-    probes = [0, 1]
-    olp, olm, orp, orm = O.probe_losses(theta, spec, seed, cfg.n_pert, cfg.eps, tok, tgt,
-                                        probes=probes, rows=sl, return_rows=True)
-    del theta
-    assert np.allclose(rows[probes, 0][:, sl], orp, rtol=1e-2)
-    assert np.allclose(rows[probes, 1][:, sl], orm, rtol=1e-2)
-    cnt = (tgt[sl] >= 0).sum()
-    glp = rows[probes, 0][:, sl].sum(axis=1) / cnt
-    glm = rows[probes, 1][:, sl].sum(axis=1) / cnt
-    assert np.allclose(glp, olp, rtol=1e-2) and np.allclose(glm, olm, rtol=1e-2)
-    assert sign_agreement(glp, glm, olp, olm) >= 0.95
-    assert estimate_cosine(spec, seed, probes, glp, glm, olp, olm) >= 0.99
-    # the full-batch losses are the means of the row sums
+    probes, sl = list(range(n_probes)), np.arange(n_rows)
+    if n_probes >= 2:
+        _row_slice_gate(cfg, theta, tok, tgt, seed, rows, probes, sl)
+    else:
+        orl, _ = native_oracle().probe_row_losses(theta, spec_of(cfg), seed, probes, cfg.eps, tok,
+                                                  tgt, rows=sl)
+        assert np.allclose(rows[probes][:, :, sl], orl, rtol=1e-2)
     n_all = (tgt >= 0).sum()
     assert np.allclose(lp, rows[:, 0].sum(axis=1) / n_all, rtol=1e-5)
     assert np.allclose(lm, rows[:, 1].sum(axis=1) / n_all, rtol=1e-5)

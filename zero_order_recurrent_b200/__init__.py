@@ -32,7 +32,7 @@ EXPORTS = (
     "zo_probe_losses_ex", "zo_coeffs", "zo_update", "zo_invalidate_shadow", "zo_step_host",
     "zo_sync_status", "zo_sign_words", "zo_status_string", "zo_kernel_launches",
     "zo_debug_cell_preact", "zo_profile", "zo_profile_read", "zo_probe_losses_static",
-    "zo_probe_losses_slice", "zo_loss", "zo_coeffs_forward",
+    "zo_probe_losses_slice", "zo_loss", "zo_coeffs_forward", "zo_debug_cell_stall",
 )
 ZO_STATIC_SCRATCH_FLOATS = 65536
 ZO_MAX_UPDATE_PROBES = 8192
@@ -83,6 +83,7 @@ def load_library(path: str = LIB_PATH):
         "zo_kernel_launches": ([], I64),
         "zo_debug_cell_preact": ([P, P, U64, I32, I32, F, P, I32, I32, P, P], ctypes.c_int),
         "zo_profile": ([P, I32], ctypes.c_int),
+        "zo_debug_cell_stall": ([P, I32, U64, P], ctypes.c_int),
         "zo_probe_losses_slice": ([P, P, U64, I32, I32, F, P, P, I32, I32, P, P, P], ctypes.c_int),
         "zo_probe_losses_static": ([ctypes.POINTER(ModelSpec), P, U64, I32, F, P, P, I32, I32, P, P,
                                     P], ctypes.c_int),
@@ -253,6 +254,12 @@ def zo_debug_cell_preact(ctx, theta, step_seed, probe0, n_probes, eps, tokens, p
     _check(load_library().zo_debug_cell_preact(
         ctx.handle, _ptr(theta), ctypes.c_uint64(step_seed), probe0, n_probes, eps, _ptr(tokens),
         B, T, _ptr(preact), _stream(stream)), "zo_debug_cell_preact")
+
+
+def zo_debug_cell_stall(ctx, kind: int, wait_ns: int, stream=None):
+    """Test hook: a tensor-core kernel whose waits all run out (include/zo_debug.h)."""
+    _check(load_library().zo_debug_cell_stall(ctx.handle, kind, ctypes.c_uint64(wait_ns),
+                                              _stream(stream)), "zo_debug_cell_stall")
 
 
 def zo_profile(ctx, enable: bool):

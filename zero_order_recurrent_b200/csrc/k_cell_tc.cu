@@ -5,21 +5,35 @@
 //   c_t = sigma(f) c_{t-1} + sigma(i) tanh(g),  h_t = sigma(o) tanh(c_t),
 // i.e. one complete forward step at Theta +- eps p_i (pith.science review,
 // "What carries the argument"; alex-wiki "Method").  The perturbed operand is
-// never stored in HBM: the bf16 shadow tile of W_l arrives by TMA, four
+// never stored in HBM: the bf16 shadow tile of W_l arrives by TMA, eight
 // generator warps add +-eps in place from the probe's Philox words, and
 // tcgen05.mma consumes it with fp32 accumulation in tensor memory.
 //
-// CTA tile: MT sub-tiles of 128 batch rows x BN gate rows (BN/4 hidden units,
-// the four gate blocks side by side so the epilogue sees i, f, g, o of a unit
-// together) x 64-deep K stages.  Warp roles (320 threads):
-//   warp 0       TMA producer (A activations, W_l tile as 4 gate boxes)
-//   warp 1       TMEM allocator and MMA issuer
-//   warps 2..9   perturbation: W tile += +-eps p in shared memory, one row
-//                per thread, two warps per SM sub-partition to hide latency
+// Tile: 256 batch rows x BN gate rows (BN/4 hidden units, the four gate blocks
+// side by side so the epilogue sees i, f, g, o of a unit together) x 64-deep K
+// stages.  Two forms:
+//   CG = 2 (cell steps and the vocabulary table): a cluster of two CTAs runs
+//     one tcgen05.mma.cta_group::2 (M = 256, N = 256) per K step.  Each CTA
+//     holds 128 of the rows of A and half of B (CTA 0 the gate rows of i and
+//     f, CTA 1 those of g and o), loads and perturbs only that half, and
+//     receives the 128 x 256 accumulator of its own rows in its tensor memory
+//     (all four gates).  An accumulator takes 256 columns, so two fit: the
+//     epilogue of one tile runs while the MMAs of the next fill the other.
+//     The MMA is issued by one thread of CTA 0; the other CTA's generator and
+//     epilogue warps arrive on CTA 0's barriers through the cluster, and MMA
+//     completion is signalled to both CTAs' barriers.
+//   CG = 1 (output layer + cross-entropy): one CTA, MT = 2 sub-tiles of 128
+//     rows, each a tcgen05.mma.cta_group::1 (M = 128).
+// Warp roles (448 threads):
+//   warp 0       TMA producer (this CTA's A rows, its gate boxes of W_l)
+//   warp 1       TMEM allocator; MMA issuer (CTA 0 of a pair)
+//   warps 2..9   perturbation: W tile += +-eps p in shared memory, two warps
+//                per SM sub-partition to hide latency
 //   warps 10..13 epilogue: TMEM -> gates -> c, h (TMEM lane quadrant = warp % 4)
 // Every mbarrier wait is bounded: past ~2 s the CTA raises an abort flag, the
 // error word gets ZO_ERR_TIMEOUT, all roles leave their loops, and tensor
-// memory is freed before exit.  No multicast form of any copy is used.
+// memory is freed before exit.  No TMA copy uses a multicast form; only the
+// MMA-completion commit is multicast to the two CTAs of a pair.
 #include <cudaTypedefs.h>
 
 #include "zo_common.cuh"
@@ -30,7 +44,7 @@ namespace zo {
 constexpr int kTcThreads = 448;
 constexpr int kGenThreads = 256;
 constexpr int kGenWarps = kGenThreads / 32;
-constexpr uint64_t kWaitLimitNs = 2000000000ull;
+constexpr uint64_t kWaitLimitNs = kDefaultWaitNs;   // default bound of a wait
 
 struct CellArgs {
   int K0;          // input width of the layer
@@ -62,6 +76,8 @@ struct CellArgs {
   int V, T, t;
   const int32_t* targets;  // [B][T]
   float* rowloss;          // [P][Bmax], accumulated
+  uint64_t wait_ns;        // bound of every mbarrier wait
+  int stall;               // test hook: the producer issues nothing (all waits run out)
 };
 
 // ---------------------------------------------------------------------------
@@ -96,6 +112,18 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+__device__ __forceinline__ bool mbar_try_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 __device__ __forceinline__ uint64_t globaltimer() {
   uint64_t t;
   asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
@@ -103,16 +131,20 @@ __device__ __forceinline__ uint64_t globaltimer() {
 }
 
 // Bounded wait.  Returns false (and raises the CTA abort flag) if the phase
-// did not complete within kWaitLimitNs, or if another role already aborted.
+// did not complete within limit_ns, or if another role already aborted.
+// CLUSTER: the barrier also receives arrivals from the other CTA of a pair
+// (acquire at cluster scope).
+template <bool CLUSTER = false>
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          unsigned* err) {
-  if (mbar_try(bar, parity)) return true;
+                                          unsigned* err, uint64_t limit_ns) {
+  auto try_once = [&] { return CLUSTER ? mbar_try_cluster(bar, parity) : mbar_try(bar, parity); };
+  if (try_once()) return true;
   const uint64_t t0 = globaltimer();
   for (uint32_t i = 1;; ++i) {
-    if (mbar_try(bar, parity)) return true;
+    if (try_once()) return true;
     if ((i & 255) == 0) {
       if (*abort_flag) return false;
-      if (globaltimer() - t0 > kWaitLimitNs) {
+      if (globaltimer() - t0 > limit_ns) {
         *abort_flag = 1;
         latch(err, kErrTimeout);
         return false;
@@ -191,6 +223,73 @@ __device__ __forceinline__ void umma_commit(uint32_t bar) {
                : "memory");
 }
 
+// ---- CTA-pair (cluster of two) forms -------------------------------------
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_id_x() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_count_x() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
+  return r;
+}
+
+// shared::cluster address of the same shared-memory offset in CTA `rank`
+__device__ __forceinline__ uint32_t peer_addr(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+
+// arrive on a barrier of the cluster (here: CTA 0's), releasing this thread's
+// earlier writes at cluster scope
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+               : "memory");
+}
+
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                   : "memory");
+}
+
+// M = 256 MMA over the pair: A rows 0..127 and B rows 0..N/2-1 from CTA 0's
+// shared memory, the rest from CTA 1's at the same offsets; each CTA's tensor
+// memory receives its own 128 rows.
+__device__ __forceinline__ void umma_bf16_pair(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                               uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// completion of this thread's earlier pair MMAs -> one arrival on the barrier
+// at offset `bar` in both CTAs of the pair
+__device__ __forceinline__ void umma_commit_pair_both(uint32_t bar) {
+  const uint16_t mask = 0x3;
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 "
+      "[%0], %1;" ::"r"(bar),
+      "h"(mask)
+      : "memory");
+}
+
+// ... or on this CTA's barrier only
+__device__ __forceinline__ void umma_commit_pair_local(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   bar)
+               : "memory");
+}
+
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
@@ -248,29 +347,35 @@ __device__ __forceinline__ TileCoord decode_tile(const CellArgs& a, int64_t tile
   return c;
 }
 
-template <int MT, int BN, int STAGES, int ACC>
+template <int MT, int BN, int STAGES, int ACC, int CG>
 struct TcCfg {
-  static constexpr int U = BN / 4;
+  static constexpr int U = BN / 4;                  // hidden units per tile
+  static constexpr int BL = BN / CG;                // gate rows of B held by this CTA
+  static constexpr int GPC = 4 / CG;                // gate blocks held by this CTA
   static constexpr int A_SUB = 128 * 128;           // one 128-row sub-tile, bytes
   static constexpr int A_BYTES = MT * A_SUB;
-  static constexpr int B_BYTES = BN * 128;
+  static constexpr int B_BYTES = BL * 128;
   static constexpr int STAGE = A_BYTES + B_BYTES;
+  static constexpr int ROWS = 128 * MT * CG;        // batch rows per tile
   static constexpr int COLS = MT * BN;              // TMEM columns per accumulator
   static constexpr int TMEM_COLS = COLS * ACC;
   static constexpr int EPI = 4 * 4 * U * 4;          // per epilogue warp: bias slice [4][U]
   static constexpr int SMEM = STAGES * STAGE + 1024 + 256 + EPI;
   static_assert(BN % 64 == 0 && BN <= 256, "BN");
+  static_assert(CG == 1 || (CG == 2 && MT == 1 && BN == 256), "pair tiles are 256 x 256");
   static_assert(TMEM_COLS == 128 || TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM columns");
+  static_assert(SMEM <= 227 * 1024, "shared memory");
 };
 
 // MODE 0: cell step.  1: output projection + cross-entropy.  2: cell step of
 // layer 0 whose input term comes from the vocabulary table (added in the
 // epilogue).  3: the vocabulary table itself (raw accumulators, no bias).
-template <int MT, int BN, int STAGES, int ACC, int MODE>
+template <int MT, int BN, int STAGES, int ACC, int MODE, int CG>
 __global__ void __launch_bounds__(kTcThreads, 1)
     cell_tc_kernel(const __grid_constant__ CUtensorMap mapA0, const __grid_constant__ CUtensorMap mapA1,
                    const __grid_constant__ CUtensorMap mapW, const CellArgs a, int P) {
-  using C = TcCfg<MT, BN, STAGES, ACC>;
+  using C = TcCfg<MT, BN, STAGES, ACC, CG>;
+  constexpr bool PAIR = CG == 2;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -289,16 +394,28 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // position in the pair (0 issues the MMAs) and the tile walk of the pair
+  const uint32_t rank = PAIR ? cluster_rank() : 0u;
+  const int64_t walker = PAIR ? (int64_t)cluster_id_x() : (int64_t)blockIdx.x;
+  const int64_t walkers = PAIR ? (int64_t)cluster_count_x() : (int64_t)gridDim.x;
+  // where generator and epilogue warps report: CTA 0's barrier (through the
+  // cluster from CTA 1)
+  auto report = [&](uint32_t bar) {
+    if (!PAIR || rank == 0)
+      mbar_arrive(bar);
+    else
+      mbar_arrive_cluster(peer_addr(bar, 0));
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(full_bar(s), 1);
-      mbar_init(ready_bar(s), kGenWarps);
+      mbar_init(ready_bar(s), kGenWarps * CG);
       mbar_init(empty_bar(s), 1);
     }
     for (int b = 0; b < ACC; ++b) {
       mbar_init(accf_bar(b), 1);
-      mbar_init(acce_bar(b), 4);
+      mbar_init(acce_bar(b), 4 * CG);
     }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -311,29 +428,39 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     prefetch_map(&mapW);
   }
   if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     smem_u32(tmem_slot)),
-                 "r"(C::TMEM_COLS)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    if constexpr (PAIR) {
+      asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                       smem_u32(tmem_slot)),
+                   "r"(C::TMEM_COLS)
+                   : "memory");
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    } else {
+      asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                       smem_u32(tmem_slot)),
+                   "r"(C::TMEM_COLS)
+                   : "memory");
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
   }
   tc_fence_before();
   __syncthreads();
+  // the other CTA's barriers are initialised before anyone arrives on them
+  if constexpr (PAIR) cluster_sync_all();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
+    if (lane == 0 && !a.stall) {
       uint32_t it = 0;
       bool ok = true;
-      for (int64_t tile = blockIdx.x; tile < a.tiles && ok; tile += gridDim.x) {
+      for (int64_t tile = walker; tile < a.tiles && ok; tile += walkers) {
         const TileCoord tc = decode_tile(a, tile, P);
-        const int row0 = tc.m * 128 * MT;
+        const int row0 = tc.m * C::ROWS + (int)rank * 128 * MT;
         for (int kb = a.kbeg; kb < a.nk; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1;
-          if (!mbar_wait(empty_bar(s), ph ^ 1, abort_flag, a.err)) {
+          if (!mbar_wait<PAIR>(empty_bar(s), ph ^ 1, abort_flag, a.err, a.wait_ns)) {
             ok = false;
             break;
           }
@@ -350,8 +477,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                           tc.ps);
           }
 #pragma unroll
-          for (int g = 0; g < 4; ++g)
-            tma_load_2d(sb + g * C::U * 128, &mapW, full_bar(s), kk, g * a.gstride + tc.n * C::U);
+          for (int gi = 0; gi < C::GPC; ++gi) {
+            const int g = (int)rank * C::GPC + gi;
+            tma_load_2d(sb + gi * C::U * 128, &mapW, full_bar(s), kk, g * a.gstride + tc.n * C::U);
+          }
         }
       }
       if (!ok) {
@@ -367,14 +496,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = umma_idesc(128, BN);
+    if (lane == 0 && rank == 0) {
+      constexpr uint32_t idesc = umma_idesc(128 * CG, BN);
       uint32_t it = 0, tcount = 0;
       bool ok = true;
-      for (int64_t tile = blockIdx.x; tile < a.tiles && ok; tile += gridDim.x, ++tcount) {
+      for (int64_t tile = walker; tile < a.tiles && ok; tile += walkers, ++tcount) {
         const int ab = tcount % ACC;
         const uint32_t aph = (tcount / ACC) & 1;
-        if (!mbar_wait(acce_bar(ab), aph ^ 1, abort_flag, a.err)) {
+        if (!mbar_wait<PAIR>(acce_bar(ab), aph ^ 1, abort_flag, a.err, a.wait_ns)) {
           ok = false;
           break;
         }
@@ -383,7 +512,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         for (int kb = a.kbeg; kb < a.nk; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1;
-          if (!mbar_wait(ready_bar(s), ph, abort_flag, a.err)) {
+          if (!mbar_wait<PAIR>(ready_bar(s), ph, abort_flag, a.err, a.wait_ns)) {
             ok = false;
             break;
           }
@@ -392,33 +521,46 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const uint64_t bdesc = umma_desc(sa + C::A_BYTES);
 #pragma unroll
           for (int k16 = 0; k16 < 4; ++k16) {
+            const uint32_t acc = (kb != a.kbeg || k16 != 0) ? 1u : 0u;
+            if constexpr (PAIR) {
+              umma_bf16_pair(dcol, umma_desc(sa) + 2 * k16, bdesc + 2 * k16, idesc, acc);
+            } else {
 #pragma unroll
-            for (int mt = 0; mt < MT; ++mt) {
-              const uint64_t adesc = umma_desc(sa + mt * C::A_SUB);
-              umma_bf16(dcol + mt * BN, adesc + 2 * k16, bdesc + 2 * k16, idesc,
-                        (kb != a.kbeg || k16 != 0) ? 1u : 0u);
+              for (int mt = 0; mt < MT; ++mt)
+                umma_bf16(dcol + mt * BN, umma_desc(sa + mt * C::A_SUB) + 2 * k16, bdesc + 2 * k16,
+                          idesc, acc);
             }
           }
-          umma_commit(empty_bar(s));
+          if constexpr (PAIR)
+            umma_commit_pair_both(empty_bar(s));
+          else
+            umma_commit(empty_bar(s));
         }
         if (!ok) break;
-        umma_commit(accf_bar(ab));
+        if constexpr (PAIR)
+          umma_commit_pair_both(accf_bar(ab));
+        else
+          umma_commit(accf_bar(ab));
       }
       // all MMAs issued by this thread complete before tensor memory is freed
-      umma_commit(drain_bar);
+      if constexpr (PAIR)
+        umma_commit_pair_local(drain_bar);
+      else
+        umma_commit(drain_bar);
       const uint64_t t0 = globaltimer();
       while (!mbar_try(drain_bar, 0) && globaltimer() - t0 < 100000000ull) {
       }
     }
   } else if (warp < 2 + kGenWarps) {
     // ------------------------------------------------------------ perturbation
-    // BN >= kGenThreads: RPT rows per thread, all 8 chunks of each row;
-    // BN <  kGenThreads: TPR threads share a row, CPT chunks each
-    constexpr int RPT = (BN + kGenThreads - 1) / kGenThreads;
-    constexpr int TPR = BN >= kGenThreads ? 1 : kGenThreads / BN;
+    // BL >= kGenThreads: RPT rows per thread, all 8 chunks of each row;
+    // BL <  kGenThreads: TPR threads share a row, CPT chunks each
+    constexpr int BL = C::BL;
+    constexpr int RPT = (BL + kGenThreads - 1) / kGenThreads;
+    constexpr int TPR = BL >= kGenThreads ? 1 : kGenThreads / BL;
     constexpr int CPT = 8 / TPR;
-    const int gt = (threadIdx.x - 64) % (BN < kGenThreads ? BN : kGenThreads);
-    const int c0 = ((threadIdx.x - 64) / (BN < kGenThreads ? BN : kGenThreads)) * CPT;
+    const int gt = (threadIdx.x - 64) % (BL < kGenThreads ? BL : kGenThreads);
+    const int c0 = ((threadIdx.x - 64) / (BL < kGenThreads ? BL : kGenThreads)) * CPT;
     const float epsf = a.eps;
     const __nv_bfloat16 eb = __float2bfloat16_rn(epsf);
     const uint32_t eps_bits = (uint32_t)(*reinterpret_cast<const uint16_t*>(&eb));
@@ -426,7 +568,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const uint32_t epsn2 = epsp2 ^ 0x80008000u;
     uint32_t it = 0;
     bool ok = true;
-    for (int64_t tile = blockIdx.x; tile < a.tiles && ok; tile += gridDim.x) {
+    for (int64_t tile = walker; tile < a.tiles && ok; tile += walkers) {
       const TileCoord tc = decode_tile(a, tile, P);
       const uint32_t probe = (uint32_t)(a.probe0 + (tc.ps >> 1));
       const uint32_t e2 = (tc.ps & 1) ? epsn2 : epsp2;
@@ -437,7 +579,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       for (int kb = a.kbeg; kb < a.nk; ++kb, ++it) {
         const int s = it % STAGES;
         const uint32_t ph = (it / STAGES) & 1;
-        if (!mbar_wait(full_bar(s), ph, abort_flag, a.err)) {
+        if (!mbar_wait(full_bar(s), ph, abort_flag, a.err, a.wait_ns)) {
           ok = false;
           break;
         }
@@ -445,8 +587,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
         for (int rr = 0; rr < RPT; ++rr) {
           const int r = gt + rr * kGenThreads;
-          if (r < BN) {
-            const int g = r / C::U, u = r % C::U;
+          if (r < BL) {
+            const int g = (int)rank * C::GPC + r / C::U, u = r % C::U;
             const int64_t R = (int64_t)g * a.gstride + (int64_t)tc.n * C::U + u;
             const int64_t j0 = a.offW + R * a.Ktot + (int64_t)kb * 64;
             const int64_t q = j0 >> 7;
@@ -474,7 +616,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         fence_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(ready_bar(s));
+        if (lane == 0) report(ready_bar(s));
       }
     }
   } else {
@@ -485,10 +627,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     float* bias_s = reinterpret_cast<float*>(smem + STAGES * C::STAGE + 256) + quad * 4 * C::U;
     uint32_t tcount = 0;
     bool ok = true;
-    for (int64_t tile = blockIdx.x; tile < a.tiles && ok; tile += gridDim.x, ++tcount) {
+    for (int64_t tile = walker; tile < a.tiles && ok; tile += walkers, ++tcount) {
       const TileCoord tc = decode_tile(a, tile, P);
       const int ab = tcount % ACC;
       const uint32_t aph = (tcount / ACC) & 1;
+      const int brow0 = tc.m * C::ROWS + (int)rank * 128 * MT;   // this CTA's first batch row
       if constexpr (MODE == 0 || MODE == 2) {
         // staged while the tile's MMAs run, so the epilogue's bias reads are
         // shared-memory broadcasts instead of one L2 round trip per chunk
@@ -504,7 +647,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // while this tile's MMAs run, pull its c_{t-1} rows (and the token's
         // vocabulary-table rows) into L2 so the epilogue's loads hit L2
         for (int mt = 0; mt < MT; ++mt) {
-          const int b = tc.m * 128 * MT + mt * 128 + rloc;
+          const int b = brow0 + mt * 128 + rloc;
           if (b < a.B) {
             prefetch_l2(a.cst + ((int64_t)tc.ps * a.Bmax + b) * a.H + tc.n * C::U,
                         C::U * (int)sizeof(float));
@@ -519,7 +662,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           }
         }
       }
-      if (!mbar_wait(accf_bar(ab), aph, abort_flag, a.err)) {
+      if (!mbar_wait<PAIR>(accf_bar(ab), aph, abort_flag, a.err, a.wait_ns)) {
         ok = false;
         break;
       }
@@ -528,7 +671,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if constexpr (MODE == 1) {
         // logits of one row live in one TMEM lane: softmax cross-entropy per row
         for (int mt = 0; mt < MT; ++mt) {
-          const int b = tc.m * 128 * MT + mt * 128 + rloc;
+          const int b = brow0 + mt * 128 + rloc;
           uint32_t z[BN];
 #pragma unroll
           for (int q = 0; q < BN / 16; ++q) {
@@ -563,7 +706,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
       } else
       for (int mt = 0; mt < MT; ++mt) {
-        const int b = tc.m * 128 * MT + mt * 128 + rloc;
+        const int b = brow0 + mt * 128 + rloc;
         const int64_t rowoff = ((int64_t)tc.ps * a.Bmax + b) * a.H;
         const bool live = b < a.B;
         const bool need_c = live && !a.first && !a.raw;
@@ -683,18 +826,26 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(acce_bar(ab));
+      if (lane == 0) report(acce_bar(ab));
     }
   }
 
   tc_fence_before();
   __syncthreads();
+  // neither CTA of a pair leaves while the other may still read its shared
+  // memory (MMA operands) or arrive on its barriers
+  if constexpr (PAIR) cluster_sync_all();
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
-                 "r"(C::TMEM_COLS)
-                 : "memory");
+    if constexpr (PAIR)
+      asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                   "r"(C::TMEM_COLS)
+                   : "memory");
+    else
+      asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                   "r"(C::TMEM_COLS)
+                   : "memory");
   }
 }
 
@@ -762,24 +913,56 @@ bool make_cell_maps(zo_ctx* c) {
   return ok;
 }
 
-template <int MT, int BN, int STAGES, int ACC, int MODE>
+template <int MT, int BN, int STAGES, int ACC, int MODE, int CG>
 static cudaError_t launch_cfg(const CUtensorMap& A0, const CUtensorMap& A1, const CUtensorMap& Wm,
                               CellArgs a, int P, int sms, cudaStream_t st) {
-  using C = TcCfg<MT, BN, STAGES, ACC>;
-  a.m_tiles = (a.B + 128 * MT - 1) / (128 * MT);
+  using C = TcCfg<MT, BN, STAGES, ACC, CG>;
+  auto kern = cell_tc_kernel<MT, BN, STAGES, ACC, MODE, CG>;
+  a.m_tiles = (a.B + C::ROWS - 1) / C::ROWS;
   a.n_tiles = MODE != 1 ? a.H / C::U : 1;
   a.tiles = (int64_t)P * a.m_tiles * a.n_tiles;
-  cudaFuncSetAttribute(cell_tc_kernel<MT, BN, STAGES, ACC, MODE>,
-                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-  const int64_t grid = a.tiles < sms ? a.tiles : sms;
-  cell_tc_kernel<MT, BN, STAGES, ACC, MODE><<<(int)grid, kTcThreads, C::SMEM, st>>>(A0, A1, Wm, a, P);
-  count_launch();
-  return cudaGetLastError();
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return e;
+  if constexpr (CG == 1) {
+    const int64_t grid = a.tiles < sms ? a.tiles : sms;
+    kern<<<(int)grid, kTcThreads, C::SMEM, st>>>(A0, A1, Wm, a, P);
+    count_launch();
+    return cudaGetLastError();
+  } else {
+    // one cluster of two CTAs per pair of SMs, as many as can be resident
+    static int max_clusters = 0;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.blockDim = dim3(kTcThreads, 1, 1);
+    cfg.dynamicSmemBytes = C::SMEM;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (max_clusters == 0) {
+      cfg.gridDim = dim3(2 * (sms / 2), 1, 1);
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) {
+        cudaGetLastError();
+        n = sms / 2;
+      }
+      max_clusters = n;
+    }
+    const int64_t clusters = a.tiles < max_clusters ? a.tiles : max_clusters;
+    cfg.gridDim = dim3((unsigned)(2 * clusters), 1, 1);
+    e = cudaLaunchKernelEx(&cfg, kern, A0, A1, Wm, a, P);
+    count_launch();
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+  }
 }
 
 cudaError_t launch_cell_tc(const zo_ctx* ctx, int layer, int t, int B, int nprobe, int probe0,
                            uint64_t seed, float eps, float* raw_out, const int32_t* tokens, int T,
-                           bool vocab, cudaStream_t st) {
+                           bool vocab, cudaStream_t st, uint64_t wait_ns, int stall) {
   const zo_model_spec& s = ctx->spec;
   const int H = s.hidden, E = s.embed;
   const int P = 2 * nprobe;
@@ -789,6 +972,8 @@ cudaError_t launch_cell_tc(const zo_ctx* ctx, int layer, int t, int B, int nprob
   const bool tab = vocab && layer == 0;
   if (tab && (t == 0 || !ctx->vt)) return cudaErrorInvalidValue;
   CellArgs a;
+  a.wait_ns = wait_ns;
+  a.stall = stall;
   a.K0 = K0;
   a.H = H;
   a.Ktot = K0 + H;
@@ -822,10 +1007,10 @@ cudaError_t launch_cell_tc(const zo_ctx* ctx, int layer, int t, int B, int nprob
   const CUtensorMap& A0 = layer == 0 ? m.x : m.h[layer - 1][t & 1];
   const CUtensorMap& A1 = m.h[layer][(t + 1) & 1];
   a.gstride = H;
-  // 256 batch rows x 256 gate rows per tile (all 512 TMEM columns): the
-  // fastest shape measured for every model size here (K from 1280 to 16384)
-  if (tab) return launch_cfg<2, 256, 3, 1, 2>(A0, A1, m.w[layer], a, P, ctx->sm_count, st);
-  return launch_cfg<2, 256, 3, 1, 0>(A0, A1, m.w[layer], a, P, ctx->sm_count, st);
+  // 256 batch rows x 256 gate rows per tile on a CTA pair, two accumulators
+  // of 256 TMEM columns per CTA, six 32 KB stages
+  if (tab) return launch_cfg<1, 256, 6, 2, 2, 2>(A0, A1, m.w[layer], a, P, ctx->sm_count, st);
+  return launch_cfg<1, 256, 6, 2, 0, 2>(A0, A1, m.w[layer], a, P, ctx->sm_count, st);
 }
 
 // Output projection + softmax cross-entropy for step t on the same
@@ -833,11 +1018,14 @@ cudaError_t launch_cell_tc(const zo_ctx* ctx, int layer, int t, int B, int nprob
 // in shared memory (V <= 64 rows, the rest zero), logits of a row in one TMEM
 // lane; rowloss[ps][b] += logsumexp(z_b) - z_b[target].
 cudaError_t launch_loss_tc(const zo_ctx* ctx, const int32_t* targets, int t, int B, int T,
-                           int nprobe, int probe0, uint64_t seed, float eps, cudaStream_t st) {
+                           int nprobe, int probe0, uint64_t seed, float eps, cudaStream_t st,
+                           uint64_t wait_ns, int stall) {
   const zo_model_spec& s = ctx->spec;
   const int H = s.hidden, L = s.layers;
   const int P = 2 * nprobe;
   CellArgs a;
+  a.wait_ns = wait_ns;
+  a.stall = stall;
   a.K0 = H;
   a.H = H;
   a.Ktot = H;
@@ -869,7 +1057,7 @@ cudaError_t launch_loss_tc(const zo_ctx* ctx, const int32_t* targets, int t, int
   a.rowloss = ctx->rowloss;
   const CellMaps& m = *ctx->maps;
   const CUtensorMap& A0 = m.h[L - 1][t & 1];
-  return launch_cfg<2, 64, 4, 2, 1>(A0, A0, m.wout, a, P, ctx->sm_count, st);
+  return launch_cfg<2, 64, 4, 2, 1, 1>(A0, A0, m.wout, a, P, ctx->sm_count, st);
 }
 
 // Vocabulary table of layer 0's input term for the chunk's probe-signs:
@@ -884,6 +1072,8 @@ cudaError_t launch_vocab_table(const zo_ctx* ctx, int nprobe, int probe0, uint64
   const int H = s.hidden, E = s.embed;
   const int P = 2 * nprobe;
   CellArgs a;
+  a.wait_ns = kWaitLimitNs;
+  a.stall = 0;
   a.K0 = E;
   a.H = H;
   a.Ktot = E + H;
@@ -914,7 +1104,7 @@ cudaError_t launch_vocab_table(const zo_ctx* ctx, int nprobe, int probe0, uint64
   a.rowloss = nullptr;
   a.gstride = H;
   const CellMaps& m = *ctx->maps;
-  return launch_cfg<2, 256, 3, 1, 3>(m.x, m.x, m.w[0], a, P, ctx->sm_count, st);
+  return launch_cfg<1, 256, 6, 2, 3, 2>(m.x, m.x, m.w[0], a, P, ctx->sm_count, st);
 }
 
 }  // namespace zo

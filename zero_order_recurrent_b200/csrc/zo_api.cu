@@ -24,6 +24,16 @@ namespace {
 
 inline cudaStream_t S(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 
+// Host-side fault injection for tests, read from the environment at every
+// call: ZO_FAULT=alloc makes zo_create's device allocations fail (it returns
+// ZO_ERR_OOM and keeps nothing allocated); ZO_FAULT=launch makes the
+// probe-loss, coefficient and update calls return ZO_ERR_CUDA before they
+// enqueue anything.  No device-side fault is ever injected.
+bool injected(const char* what) {
+  const char* f = getenv("ZO_FAULT");
+  return f && strcmp(f, what) == 0;
+}
+
 #define ZO_CUDA(call)                      \
   do {                                     \
     cudaError_t e_ = (call);               \
@@ -167,8 +177,13 @@ int zo_create(const zo_model_spec* spec, zo_ctx** out) {
   build_segments(s, c->seg);
   const int64_t B = s.max_batch, E = s.embed, H = s.hidden, V = s.vocab, L = s.layers;
   int rc = ZO_OK;
+  const bool fail_alloc = injected("alloc");
   auto alloc = [&](void** p, size_t bytes) {
     if (rc != ZO_OK) return;
+    if (fail_alloc) {
+      rc = ZO_ERR_OOM;
+      return;
+    }
     if (cudaMalloc(p, bytes) != cudaSuccess) {
       cudaGetLastError();
       rc = ZO_ERR_OOM;
@@ -305,6 +320,7 @@ static int probe_losses_range(zo_ctx* ctx, const float* theta, uint64_t seed, in
     return ZO_ERR_INVALID_ARG;
   if (batch < 1 || batch > ctx->spec.max_batch || seq < 1 || seq > ctx->spec.max_seq)
     return ZO_ERR_INVALID_ARG;
+  if (injected("launch")) return ZO_ERR_CUDA;
   cudaStream_t st = S(stream);
   const int B = batch, T = seq;
   const int64_t Vv = ctx->spec.vocab, Ee = ctx->spec.embed, Hh = ctx->spec.hidden;
@@ -404,6 +420,7 @@ int zo_coeffs(zo_ctx* ctx, const float* lp, const float* lm, int32_t n, float ep
               float* coeffs, void* stream) {
   if (!ctx || !lp || !lm || !coeffs || n < 1) return ZO_ERR_INVALID_ARG;
   if (!(eps > 0.f) || !isfinite(eps) || !isfinite(eta)) return ZO_ERR_INVALID_ARG;
+  if (injected("launch")) return ZO_ERR_CUDA;
   ZO_CUDA(timed(ctx, S(stream), ZO_KIND_OTHER, 0.0, 0.0, [&] {
     return launch_coeffs(lp, lm, n, eps, eta, coeffs, ctx->err, S(stream));
   }));
@@ -430,6 +447,7 @@ int zo_coeffs_forward(zo_ctx* ctx, const float* lp, const float* l0, int32_t n, 
 int zo_update(zo_ctx* ctx, float* theta, uint64_t seed, int32_t n, const float* coeffs,
               void* stream) {
   if (!ctx || !theta || !coeffs || n < 1 || n > ZO_MAX_UPDATE_PROBES) return ZO_ERR_INVALID_ARG;
+  if (injected("launch")) return ZO_ERR_CUDA;
   __nv_bfloat16* sh = ctx->spec.dtype == ZO_DTYPE_BF16 ? ctx->shadow : nullptr;
   const double bytes = (double)ctx->seg.d_pad * (sh ? 10.0 : 8.0);
   ZO_CUDA(timed(ctx, S(stream), ZO_KIND_UPDATE, 0.0, bytes,
@@ -529,6 +547,20 @@ int zo_profile_read(zo_ctx* ctx, int32_t kind, int64_t* launches, double* total_
   if (total_ms) *total_ms = ms;
   if (total_flops) *total_flops = fl;
   if (total_bytes) *total_bytes = by;
+  return ZO_OK;
+}
+
+int zo_debug_cell_stall(zo_ctx* ctx, int32_t kind, uint64_t wait_ns, void* stream) {
+  if (!ctx || (kind != 0 && kind != 1) || wait_ns < 1000ull || wait_ns > 10000000000ull)
+    return ZO_ERR_INVALID_ARG;
+  if (ctx->spec.dtype != ZO_DTYPE_BF16) return ZO_ERR_UNSUPPORTED;
+  cudaStream_t st = S(stream);
+  const int B = ctx->spec.max_batch, T = ctx->spec.max_seq;
+  if (kind == 0)
+    ZO_CUDA(launch_cell_tc(ctx, 0, 1, B, 1, 0, 0, 1e-3f, nullptr, ctx->tok, T, false, st, wait_ns,
+                           1));
+  else
+    ZO_CUDA(launch_loss_tc(ctx, ctx->tgt, 0, B, T, 1, 0, 0, 1e-3f, st, wait_ns, 1));
   return ZO_OK;
 }
 

@@ -117,11 +117,17 @@ cudaError_t launch_perturb_small(const zo_ctx* ctx, const float* theta, uint64_t
                                  int nprobe, float eps, cudaStream_t st);
 cudaError_t launch_gather_x(const zo_ctx* ctx, const int32_t* tokens, int t, int B, int T,
                             int nprobe, cudaStream_t st);
+// wait_ns bounds every mbarrier wait of the launch; stall = 1 (a test hook)
+// makes the producer issue nothing, so every wait runs out and the kernel
+// latches ZO_ERR_TIMEOUT with no copy or MMA in flight
+constexpr uint64_t kDefaultWaitNs = 2000000000ull;
 cudaError_t launch_loss_tc(const zo_ctx* ctx, const int32_t* targets, int t, int B, int T,
-                           int nprobe, int probe0, uint64_t seed, float eps, cudaStream_t st);
+                           int nprobe, int probe0, uint64_t seed, float eps, cudaStream_t st,
+                           uint64_t wait_ns = kDefaultWaitNs, int stall = 0);
 cudaError_t launch_cell_tc(const zo_ctx* ctx, int layer, int t, int B, int nprobe, int probe0,
                            uint64_t seed, float eps, float* raw_out, const int32_t* tokens, int T,
-                           bool vocab, cudaStream_t st);
+                           bool vocab, cudaStream_t st, uint64_t wait_ns = kDefaultWaitNs,
+                           int stall = 0);
 // vocabulary table (rows kVocabRows per probe-sign) and the first step of
 // layer 0 from it
 constexpr int kVocabRows = 64;

@@ -31,13 +31,16 @@ def gather_losses(lp_local: torch.Tensor, lm_local: torch.Tensor, n_pert: int, g
     world = dist.get_world_size(group)
     counts = [probe_slice(n_pert, r, world)[1] for r in range(world)]
     m = max(counts)
-    mine = torch.zeros(2, m, dtype=lp_local.dtype, device=lp_local.device)
-    mine[0, :lp_local.numel()] = lp_local
-    mine[1, :lm_local.numel()] = lm_local
+    dev = lp_local.device
+    # gloo gathers host tensors: device slices travel through host memory
+    via = torch.device("cpu") if dist.get_backend(group) == "gloo" else dev
+    mine = torch.zeros(2, m, dtype=lp_local.dtype, device=via)
+    mine[0, :lp_local.numel()] = lp_local.to(via)
+    mine[1, :lm_local.numel()] = lm_local.to(via)
     parts = [torch.empty_like(mine) for _ in range(world)]
     dist.all_gather(parts, mine, group=group)
-    lp = torch.cat([p[0, :c] for p, c in zip(parts, counts)])
-    lm = torch.cat([p[1, :c] for p, c in zip(parts, counts)])
+    lp = torch.cat([p[0, :c] for p, c in zip(parts, counts)]).to(dev)
+    lm = torch.cat([p[1, :c] for p, c in zip(parts, counts)]).to(dev)
     return lp, lm
 
 

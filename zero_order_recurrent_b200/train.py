@@ -30,9 +30,15 @@ def _repo_root():
 def train(task: str = "copy", steps: int = 1000, n_pert: int = 64, eps: float = 1e-3,
           eta: float = 1e-3, batch: int = 8, max_len: int = 10, eval_lengths=(11, 20, 40, 60),
           embed: int = 16, hidden: int = 32, layers: int = 1, seed: int = 0,
-          log_every: int = 100, theta=None, estimator: str = "central"):
-    """Runs `steps` zero-order updates; returns the loss history, the evaluation
-    losses per length, the device time per step and the final theta (device).
+          log_every: int = 100, theta=None, estimator: str = "central", start_step: int = 0,
+          checkpoint: str = None, checkpoint_every: int = 0):
+    """Runs zero-order updates start_step .. steps-1; returns the loss history,
+    the evaluation losses per length, the device time per step and the final
+    theta (device).  Each step's batch and probes depend only on (seed, step),
+    so a run resumed from a checkpoint (theta and start_step, see
+    checkpoint.py) repeats the uninterrupted run exactly; with `checkpoint`
+    set, theta and the next step are saved every `checkpoint_every` steps and
+    at the end.
     estimator "central": c_i = eta (L+_i - L-_i)/(2 eps n) (CD-RGE);
     "forward": c_i = eta (L+_i - L(theta))/(eps n) with L(theta) from zo_loss."""
     if estimator not in ("central", "forward"):
@@ -54,12 +60,12 @@ def train(task: str = "copy", steps: int = 1000, n_pert: int = 64, eps: float = 
     lm = torch.empty(n_pert, device=dev)
     coef = torch.empty(n_pert, device=dev)
     l0 = torch.empty(1, device=dev)
-    rng = np.random.default_rng(seed)
+    from zero_order_recurrent_b200 import checkpoint as ckpt
     history = []
     ms = 0.0
     with zo.Context(V, embed, hidden, layers, "f32", batch, T_eval, 0) as ctx:
-        for step in range(steps):
-            lengths = rng.integers(1, max_len + 1, size=batch)
+        for step in range(start_step, steps):
+            lengths = np.random.default_rng((seed, 7, step)).integers(1, max_len + 1, size=batch)
             tok, tgt = W.transduction_batch(task, lengths, T_train, seed=seed * 1000003 + step)
             tok_d = torch.from_numpy(tok).to(dev)
             tgt_d = torch.from_numpy(tgt).to(dev)
@@ -83,6 +89,10 @@ def train(task: str = "copy", steps: int = 1000, n_pert: int = 64, eps: float = 
                 history.append((step, float(((lp + lm) * 0.5).mean())))
             torch.cuda.synchronize()
             ms += e0.elapsed_time(e1)
+            if checkpoint and ((checkpoint_every and (step + 1) % checkpoint_every == 0)
+                               or step == steps - 1):
+                ckpt.save(checkpoint, theta, step + 1, seed, task=task, n_pert=n_pert, eps=eps,
+                          eta=eta, estimator=estimator)
         evals = {}
         for L in eval_lengths:
             tok, tgt = W.transduction_batch(task, [L] * batch, W.task_length(task, L),
@@ -97,7 +107,7 @@ def train(task: str = "copy", steps: int = 1000, n_pert: int = 64, eps: float = 
     return {"task": task, "estimator": estimator, "steps": steps, "n_pert": n_pert, "eps": eps,
             "eta": eta,
             "max_len": max_len, "history": history, "eval": evals,
-            "ms_per_step": ms / max(steps, 1), "theta": theta}
+            "ms_per_step": ms / max(steps - start_step, 1), "theta": theta}
 
 
 def main(argv=None):
@@ -115,12 +125,26 @@ def main(argv=None):
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--log-every", type=int, default=100)
     ap.add_argument("--estimator", default="central", choices=["central", "forward"])
+    ap.add_argument("--checkpoint", default=None, help="save theta and the next step here")
+    ap.add_argument("--checkpoint-every", type=int, default=0)
+    ap.add_argument("--resume", default=None, help="start from this checkpoint")
     args = ap.parse_args(argv)
+    theta0, start = None, 0
+    if args.resume:
+        import torch
+
+        from zero_order_recurrent_b200 import checkpoint as ckpt
+        th, start, run_seed, _ = ckpt.load(args.resume)
+        if run_seed != args.seed:
+            raise SystemExit(f"checkpoint is of run seed {run_seed}, not {args.seed}")
+        theta0 = torch.from_numpy(th).cuda()
     for eta in args.eta:
         r = train(task=args.task, steps=args.steps, n_pert=args.n_pert, eps=args.eps, eta=eta,
                   batch=args.batch, max_len=args.max_len, eval_lengths=args.eval_lengths,
                   hidden=args.hidden, seed=args.seed, log_every=args.log_every,
-                  estimator=args.estimator)
+                  estimator=args.estimator, theta=None if theta0 is None else theta0.clone(),
+                  start_step=start, checkpoint=args.checkpoint,
+                  checkpoint_every=args.checkpoint_every)
         r.pop("theta")
         print(json.dumps(r), flush=True)
 
