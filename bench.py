@@ -38,6 +38,7 @@ import numpy as np  # noqa: E402
 import workloads as W  # noqa: E402
 
 METRIC = "CD-RGE steps/s and perturbed-forward tokens/s on 1 B200; % of roofline"
+CELL_VARIANTS = {"perturbed-operand": 0, "exact-eps": 1, "direct-w": 2}
 L2_BYTES = 126 * 1024 * 1024
 CLOCK_QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
                "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -161,6 +162,8 @@ def run_ours(args, cfg):
     coef = torch.empty(n, device=dev)
     flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
     ctx = zo.Context.for_config(cfg)
+    if args.cell_variant != "perturbed-operand":
+        zo.zo_debug_cell_variant(ctx, CELL_VARIANTS[args.cell_variant])
     st = torch.cuda.current_stream()
 
     def step(k):
@@ -417,6 +420,11 @@ def main():
                     help="probes per pass (default: the workload's); smaller chunks hold less "
                          "workspace, e.g. for a profiler capture")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cell-variant", default="perturbed-operand", choices=sorted(CELL_VARIANTS),
+                    help="how the cell GEMMs form W +- eps P (include/zo_debug.h): the bf16 tile "
+                         "perturbed in shared memory after a TMA load (default), the separate "
+                         "+-eps P product (exact eps, twice the MMA work), or the tile read into "
+                         "registers and perturbed there")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -435,6 +443,8 @@ def main():
                               if world > 1 else "single GPU"),
               "l2": "flushed (256 MB write) before every timed step, flush untimed",
               "tokens": "seeded synthetic (workloads module)"}
+    if args.cell_variant != "perturbed-operand":
+        config["cell_variant"] = args.cell_variant
     dtype = "bf16" if cfg.dtype == "bf16" else "f32"
 
     if args.impl == "reference":

@@ -39,6 +39,30 @@ extern "C" {
  */
 ZO_API int zo_debug_cell_stall(zo_ctx* ctx, int32_t kind, uint64_t wait_ns, void* stream);
 
+/*
+ * zo_debug_cell_variant selects, for the ZO_DTYPE_BF16 context's later calls,
+ * how the tensor-core cell GEMMs apply the perturbation (the weights at
+ * Theta +- eps p_i: alex-wiki "Method"; pith.science review, "What carries
+ * the argument").  Every variant computes the same forward; they differ in
+ * rounding and speed:
+ *   ZO_CELL_PERTURBED_OPERAND (0, default)  B = bf16(bf16(W) +- bf16(eps) p),
+ *       the bf16 tile of W staged in shared memory by TMA and perturbed there;
+ *   ZO_CELL_EXACT_EPS (1)  G = A bf16(W)^T + A (+-bf16(eps) p)^T, the two
+ *       products accumulated in fp32: the perturbation is not lost in the
+ *       rounding of bf16(W) +- eps; twice the MMA work;
+ *   ZO_CELL_DIRECT_W (2)  B as in 0, but the generator warps read the bf16
+ *       rows of W from global memory into registers and store the perturbed
+ *       tile into shared memory themselves (one shared-memory pass instead of
+ *       three).
+ * Embedding rows and biases are perturbed in fp32 in every variant.  Returns
+ * ZO_ERR_UNSUPPORTED for ZO_DTYPE_FP32 contexts, ZO_ERR_INVALID_ARG for an
+ * unknown variant.  Synchronous, host only.
+ */
+#define ZO_CELL_PERTURBED_OPERAND 0
+#define ZO_CELL_EXACT_EPS 1
+#define ZO_CELL_DIRECT_W 2
+ZO_API int zo_debug_cell_variant(zo_ctx* ctx, int32_t variant);
+
 ZO_API int zo_debug_cell_preact(zo_ctx* ctx, const float* theta_dev, uint64_t step_seed,
                                 int32_t probe0, int32_t n_probes, float eps,
                                 const int32_t* tokens_dev, int32_t batch, int32_t seq,

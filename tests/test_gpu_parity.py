@@ -356,9 +356,12 @@ def _bf16(x):
 
 
 @pytest.mark.parametrize("B,E,H", [(200, 64, 64), (128, 128, 128), (300, 256, 1024)])
-def test_tc_cell_preactivation_matches_emulation(B, E, H):
+@pytest.mark.parametrize("xp", [0, 1, 2], ids=["perturbed_operand", "exact_eps", "direct_w"])
+def test_tc_cell_preactivation_matches_emulation(B, E, H, xp):
     """One tensor-core cell step (layer 0, t = 0) against an fp64 evaluation of
-    the same bf16 operands: x = bf16(E +- eps p), W = bf16(bf16(W) +- bf16(eps) p)."""
+    the same bf16 operands: x = bf16(E +- eps p) and either
+    W = bf16(bf16(W) +- bf16(eps) p) or, with the exact-eps variant, the sum of
+    the products with bf16(W) and with +-bf16(eps) p."""
     V, n = 50, 2
     cfg = W.small_config(vocab=V, embed=E, hidden=H, layers=1, dtype="bf16")
     theta = W.init_theta(cfg, seed=8)
@@ -368,6 +371,7 @@ def test_tc_cell_preactivation_matches_emulation(B, E, H):
     segs, _ = O.layout(V, E, H, 1)
     offE, offW, offb = segs[0][3], segs[1][3], segs[2][3]
     with zo.Context(V, E, H, 1, "bf16", B, 1, n) as ctx:
+        zo.zo_debug_cell_variant(ctx, xp)
         out = torch.full((2 * n, B, 4 * H), float("nan"), device="cuda")
         zo.zo_debug_cell_preact(ctx, dev(theta), seed, 0, n, float(eps), dev(tok), out)
         assert zo.zo_sync_status(ctx) == zo.ZO_OK
@@ -379,7 +383,11 @@ def test_tc_cell_preactivation_matches_emulation(B, E, H):
         pb = O.probe_signs(seed, i, offb, 4 * H).astype(np.float32)
         for s, sg in ((0, 1.0), (1, -1.0)):
             x = _bf16((theta[offE:offE + V * E].reshape(V, E) + np.float32(sg) * eps * pE)[tok[:, 0]])
-            Wp = _bf16(_bf16(Wt) + np.float32(sg) * _bf16(np.float32(eps)) * pW)
+            if xp == 1:
+                Wp = _bf16(Wt).astype(np.float64) + \
+                    float(sg) * float(_bf16(np.float32(eps))) * pW.astype(np.float64)
+            else:
+                Wp = _bf16(_bf16(Wt) + np.float32(sg) * _bf16(np.float32(eps)) * pW)
             bias = (theta[offb:offb + 4 * H] + np.float32(sg) * eps * pb).astype(np.float64)
             want = x.astype(np.float64) @ Wp.astype(np.float64).T + bias
             g = got[2 * i + s]
@@ -388,13 +396,16 @@ def test_tc_cell_preactivation_matches_emulation(B, E, H):
                 (i, s, float(err.max()))
 
 
-@pytest.mark.parametrize("V,E,H,L,B,T,n", [(50, 64, 64, 2, 200, 4, 4), (50, 128, 256, 1, 128, 3, 3)])
-def test_bf16_small_matches_oracle(V, E, H, L, B, T, n):
+@pytest.mark.parametrize("xp", [0, 1, 2], ids=["perturbed_operand", "exact_eps", "direct_w"])
+@pytest.mark.parametrize("V,E,H,L,B,T,n", [(50, 64, 64, 2, 200, 4, 4), (50, 128, 256, 1, 128, 3, 3),
+                                           (50, 512, 64, 2, 256, 3, 2)])
+def test_bf16_small_matches_oracle(V, E, H, L, B, T, n, xp):
     cfg = W.small_config(vocab=V, embed=E, hidden=H, layers=L, dtype="bf16")
     theta = W.init_theta(cfg, seed=1)
     tok, tgt = W.markov_batch(B, T, step=0, vocab=V)
     seed = W.step_seed(3)
     with zo.Context(V, E, H, L, "bf16", B, T, n) as ctx:
+        zo.zo_debug_cell_variant(ctx, xp)
         lp, lm, rows = gpu_losses(ctx, theta, seed, n, 1e-3, tok, tgt, rows=True)
     olp, olm, orp, orm = O.probe_losses(theta, (V, E, H, L), seed, n, 1e-3, tok, tgt, return_rows=True)
     assert np.allclose(lp, olp, rtol=1e-2) and np.allclose(lm, olm, rtol=1e-2)

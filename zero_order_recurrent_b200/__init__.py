@@ -33,7 +33,9 @@ EXPORTS = (
     "zo_sync_status", "zo_sign_words", "zo_status_string", "zo_kernel_launches",
     "zo_debug_cell_preact", "zo_profile", "zo_profile_read", "zo_probe_losses_static",
     "zo_probe_losses_slice", "zo_loss", "zo_coeffs_forward", "zo_debug_cell_stall",
+    "zo_debug_cell_variant",
 )
+ZO_CELL_PERTURBED_OPERAND, ZO_CELL_EXACT_EPS, ZO_CELL_DIRECT_W = 0, 1, 2
 ZO_STATIC_SCRATCH_FLOATS = 65536
 ZO_MAX_UPDATE_PROBES = 8192
 ZO_KIND_CELL, ZO_KIND_LOSS, ZO_KIND_UPDATE, ZO_KIND_OTHER = 0, 1, 2, 3
@@ -84,6 +86,7 @@ def load_library(path: str = LIB_PATH):
         "zo_debug_cell_preact": ([P, P, U64, I32, I32, F, P, I32, I32, P, P], ctypes.c_int),
         "zo_profile": ([P, I32], ctypes.c_int),
         "zo_debug_cell_stall": ([P, I32, U64, P], ctypes.c_int),
+        "zo_debug_cell_variant": ([P, I32], ctypes.c_int),
         "zo_probe_losses_slice": ([P, P, U64, I32, I32, F, P, P, I32, I32, P, P, P], ctypes.c_int),
         "zo_probe_losses_static": ([ctypes.POINTER(ModelSpec), P, U64, I32, F, P, P, I32, I32, P, P,
                                     P], ctypes.c_int),
@@ -260,6 +263,11 @@ def zo_debug_cell_stall(ctx, kind: int, wait_ns: int, stream=None):
     """Test hook: a tensor-core kernel whose waits all run out (include/zo_debug.h)."""
     _check(load_library().zo_debug_cell_stall(ctx.handle, kind, ctypes.c_uint64(wait_ns),
                                               _stream(stream)), "zo_debug_cell_stall")
+
+
+def zo_debug_cell_variant(ctx, variant: int):
+    """How the cell GEMMs form the perturbed operand (ZO_CELL_*, include/zo_debug.h)."""
+    _check(load_library().zo_debug_cell_variant(ctx.handle, int(variant)), "zo_debug_cell_variant")
 
 
 def zo_profile(ctx, enable: bool):

@@ -76,6 +76,7 @@ struct CellArgs {
   int V, T, t;
   const int32_t* targets;  // [B][T]
   float* rowloss;          // [P][Bmax], accumulated
+  const __nv_bfloat16* wsh;  // bf16 shadow of W_l (row stride Ktot), read directly with GB
   uint64_t wait_ns;        // bound of every mbarrier wait
   int stall;               // test hook: the producer issues nothing (all waits run out)
 };
@@ -370,7 +371,19 @@ struct TcCfg {
 // MODE 0: cell step.  1: output projection + cross-entropy.  2: cell step of
 // layer 0 whose input term comes from the vocabulary table (added in the
 // epilogue).  3: the vocabulary table itself (raw accumulators, no bias).
-template <int MT, int BN, int STAGES, int ACC, int MODE, int CG>
+// XP = 1 (MODE 0, 2, 3): the perturbation as a product of its own,
+// G = A W^T + A (+-eps P)^T - the K stages run twice, first over the bf16
+// shadow tiles of W untouched, then over tiles the generator warps fill with
+// +-bf16(eps) p (only A is loaded for those), both into one accumulator - so
+// the +- pair differs by exactly the eps term instead of by the rounding of
+// bf16(theta) +- eps.  Twice the MMA work of XP = 0.
+//
+// GB = 1 (pair tiles, XP = 0): the generator warps read their rows of the W
+// tile straight from global memory into registers, three stages ahead, add
+// +-eps p there and store the perturbed tile into shared memory (swizzled);
+// only A arrives by TMA.  The W tile then crosses shared memory once (the
+// store) instead of three times (TMA write, load, store).
+template <int MT, int BN, int STAGES, int ACC, int MODE, int CG, int XP = 0, int GB = 0>
 __global__ void __launch_bounds__(kTcThreads, 1)
     cell_tc_kernel(const __grid_constant__ CUtensorMap mapA0, const __grid_constant__ CUtensorMap mapA1,
                    const __grid_constant__ CUtensorMap mapW, const CellArgs a, int P) {
@@ -398,6 +411,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const uint32_t rank = PAIR ? cluster_rank() : 0u;
   const int64_t walker = PAIR ? (int64_t)cluster_id_x() : (int64_t)blockIdx.x;
   const int64_t walkers = PAIR ? (int64_t)cluster_count_x() : (int64_t)gridDim.x;
+  // K stages of a tile (twice over with XP: W, then +-eps P)
+  const int kend = XP ? 2 * a.nk - a.kbeg : a.nk;
   // where generator and epilogue warps report: CTA 0's barrier (through the
   // cluster from CTA 1)
   auto report = [&](uint32_t bar) {
@@ -457,17 +472,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       for (int64_t tile = walker; tile < a.tiles && ok; tile += walkers) {
         const TileCoord tc = decode_tile(a, tile, P);
         const int row0 = tc.m * C::ROWS + (int)rank * 128 * MT;
-        for (int kb = a.kbeg; kb < a.nk; ++kb, ++it) {
+        for (int kb = a.kbeg; kb < kend; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1;
           if (!mbar_wait<PAIR>(empty_bar(s), ph ^ 1, abort_flag, a.err, a.wait_ns)) {
             ok = false;
             break;
           }
-          mbar_expect_tx(full_bar(s), C::STAGE);
+          const bool pstage = XP && kb >= a.nk;   // a +-eps P stage: A only
+          mbar_expect_tx(full_bar(s), (pstage || GB) ? C::A_BYTES : C::STAGE);
           const uint32_t sa = sbase + s * C::STAGE;
           const uint32_t sb = sa + C::A_BYTES;
-          const int kk = kb * 64;
+          const int kk = (pstage ? kb - a.nk + a.kbeg : kb) * 64;
 #pragma unroll
           for (int mt = 0; mt < MT; ++mt) {
             if (kk < a.K0)
@@ -476,10 +492,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               tma_load_3d(sa + mt * C::A_SUB, &mapA1, full_bar(s), kk - a.K0, row0 + mt * 128,
                           tc.ps);
           }
+          if (!pstage && !GB) {
 #pragma unroll
-          for (int gi = 0; gi < C::GPC; ++gi) {
-            const int g = (int)rank * C::GPC + gi;
-            tma_load_2d(sb + gi * C::U * 128, &mapW, full_bar(s), kk, g * a.gstride + tc.n * C::U);
+            for (int gi = 0; gi < C::GPC; ++gi) {
+              const int g = (int)rank * C::GPC + gi;
+              tma_load_2d(sb + gi * C::U * 128, &mapW, full_bar(s), kk,
+                          g * a.gstride + tc.n * C::U);
+            }
           }
         }
       }
@@ -509,7 +528,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         tc_fence_after();
         const uint32_t dcol = tmem_base + ab * C::COLS;
-        for (int kb = a.kbeg; kb < a.nk; ++kb, ++it) {
+        for (int kb = a.kbeg; kb < kend; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1;
           if (!mbar_wait<PAIR>(ready_bar(s), ph, abort_flag, a.err, a.wait_ns)) {
@@ -568,7 +587,87 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const uint32_t epsn2 = epsp2 ^ 0x80008000u;
     uint32_t it = 0;
     bool ok = true;
-    for (int64_t tile = walker; tile < a.tiles && ok; tile += walkers) {
+    if constexpr (GB) {
+      // this thread: row r = gt of the CTA's B half, chunks c0 .. c0 + 3 (64
+      // contiguous bytes of the row's 128-byte K slice)
+      static_assert(PAIR && XP == 0 && RPT == 1 && CPT == 4, "direct W loads: pair tiles");
+      constexpr int D = 3;                           // stages of loads in flight
+      const int r = gt;
+      const int g = (int)rank * C::GPC + r / C::U, u = r % C::U;
+      const int64_t Rbase = (int64_t)g * a.gstride + u;
+      uint4 buf[D][CPT];
+      // load cursor: (tile, K stage) of the next loads, D stages ahead
+      int64_t ltile = walker;
+      int lkb = a.kbeg;
+      auto issue = [&](uint4 (&dst)[CPT]) {
+        if (ltile < a.tiles) {
+          const TileCoord lt = decode_tile(a, ltile, P);
+          const uint4* src = reinterpret_cast<const uint4*>(
+              a.wsh + (Rbase + (int64_t)lt.n * C::U) * a.Ktot + (int64_t)lkb * 64 + c0 * 8);
+#pragma unroll
+          for (int cc = 0; cc < CPT; ++cc) dst[cc] = __ldg(src + cc);
+          if (++lkb == a.nk) {
+            lkb = a.kbeg;
+            ltile += walkers;
+          }
+        }
+      };
+#pragma unroll
+      for (int d = 0; d < D; ++d) issue(buf[d]);
+      int64_t ctile = walker;
+      int ckb = a.kbeg;
+      TileCoord ct = decode_tile(a, ctile < a.tiles ? ctile : 0, P);
+      int64_t cq = -1;
+      uint4 cw = make_uint4(0u, 0u, 0u, 0u);
+      while (ok && ctile < a.tiles) {
+#pragma unroll
+        for (int d = 0; d < D; ++d) {
+          if (ok && ctile < a.tiles) {
+            const int s = it % STAGES;
+            const uint32_t ph = (it / STAGES) & 1;
+            if (!mbar_wait(full_bar(s), ph, abort_flag, a.err, a.wait_ns)) {
+              ok = false;
+            } else {
+              const uint32_t probe = (uint32_t)(a.probe0 + (ct.ps >> 1));
+              const uint32_t e2 = (ct.ps & 1) ? epsn2 : epsp2;
+              const int64_t R = Rbase + (int64_t)ct.n * C::U;
+              const int64_t j0 = a.offW + R * a.Ktot + (int64_t)ckb * 64;
+              const int64_t q = j0 >> 7;
+              if (q != cq) {
+                cw = sign_block(a.seed, probe, (uint64_t)q);
+                cq = q;
+              }
+              const bool upper = (j0 >> 6) & 1;
+              const uint32_t wsel = c0 < 4 ? (upper ? cw.z : cw.x) : (upper ? cw.w : cw.y);
+              uint8_t* row = smem + s * C::STAGE + C::A_BYTES + r * 128;
+#pragma unroll
+              for (int cc = 0; cc < CPT; ++cc) {
+                const int c16 = c0 + cc;
+                const uint32_t w = wsel >> (4 * (c16 & 3));
+                uint4 v = buf[d][cc];
+                v.x = bf16x2_add(v.x, ((w << 15) & 0x80008000u) ^ e2);
+                v.y = bf16x2_add(v.y, ((w << 14) & 0x80008000u) ^ e2);
+                v.z = bf16x2_add(v.z, ((w << 13) & 0x80008000u) ^ e2);
+                v.w = bf16x2_add(v.w, ((w << 12) & 0x80008000u) ^ e2);
+                *reinterpret_cast<uint4*>(row + ((c16 ^ (r & 7)) << 4)) = v;
+              }
+              fence_async_smem();
+              __syncwarp();
+              if (lane == 0) report(ready_bar(s));
+              issue(buf[d]);
+              ++it;
+              if (++ckb == a.nk) {
+                ckb = a.kbeg;
+                ctile += walkers;
+                cq = -1;
+                if (ctile < a.tiles) ct = decode_tile(a, ctile, P);
+              }
+            }
+          }
+        }
+      }
+    }
+    for (int64_t tile = walker; tile < a.tiles && ok && !GB; tile += walkers) {
       const TileCoord tc = decode_tile(a, tile, P);
       const uint32_t probe = (uint32_t)(a.probe0 + (tc.ps >> 1));
       const uint32_t e2 = (tc.ps & 1) ? epsn2 : epsp2;
@@ -576,7 +675,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       uint4 cw[RPT];
 #pragma unroll
       for (int rr = 0; rr < RPT; ++rr) cq[rr] = -1;
-      for (int kb = a.kbeg; kb < a.nk; ++kb, ++it) {
+      for (int kb = a.kbeg; kb < kend; ++kb, ++it) {
         const int s = it % STAGES;
         const uint32_t ph = (it / STAGES) & 1;
         if (!mbar_wait(full_bar(s), ph, abort_flag, a.err, a.wait_ns)) {
@@ -584,13 +683,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           break;
         }
         uint8_t* tileB = smem + s * C::STAGE + C::A_BYTES;
+        // XP: W stages go to the MMA as loaded; +-eps P stages are written here
+        const bool wstage = XP && kb < a.nk;
+        const int kbk = XP && kb >= a.nk ? kb - a.nk + a.kbeg : kb;
 #pragma unroll
         for (int rr = 0; rr < RPT; ++rr) {
           const int r = gt + rr * kGenThreads;
-          if (r < BL) {
+          if (r < BL && !wstage) {
             const int g = (int)rank * C::GPC + r / C::U, u = r % C::U;
             const int64_t R = (int64_t)g * a.gstride + (int64_t)tc.n * C::U + u;
-            const int64_t j0 = a.offW + R * a.Ktot + (int64_t)kb * 64;
+            const int64_t j0 = a.offW + R * a.Ktot + (int64_t)kbk * 64;
             const int64_t q = j0 >> 7;
             if (q != cq[rr]) {
               cw[rr] = sign_block(a.seed, probe, (uint64_t)q);
@@ -604,13 +706,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             for (int cc = 0; cc < CPT; ++cc) {
               const int c16 = c0 + cc;
               uint4* p = reinterpret_cast<uint4*>(row + ((c16 ^ (r & 7)) << 4));
-              uint4 v = *p;
               const uint32_t w = (c16 < 4 ? wlo : whi) >> (4 * (c16 & 3));
-              v.x = bf16x2_add(v.x, ((w << 15) & 0x80008000u) ^ e2);
-              v.y = bf16x2_add(v.y, ((w << 14) & 0x80008000u) ^ e2);
-              v.z = bf16x2_add(v.z, ((w << 13) & 0x80008000u) ^ e2);
-              v.w = bf16x2_add(v.w, ((w << 12) & 0x80008000u) ^ e2);
-              *p = v;
+              if (XP) {
+                // the +-eps p tile itself
+                *p = make_uint4(((w << 15) & 0x80008000u) ^ e2, ((w << 14) & 0x80008000u) ^ e2,
+                                ((w << 13) & 0x80008000u) ^ e2, ((w << 12) & 0x80008000u) ^ e2);
+              } else {
+                uint4 v = *p;
+                v.x = bf16x2_add(v.x, ((w << 15) & 0x80008000u) ^ e2);
+                v.y = bf16x2_add(v.y, ((w << 14) & 0x80008000u) ^ e2);
+                v.z = bf16x2_add(v.z, ((w << 13) & 0x80008000u) ^ e2);
+                v.w = bf16x2_add(v.w, ((w << 12) & 0x80008000u) ^ e2);
+                *p = v;
+              }
             }
           }
         }
@@ -913,11 +1021,11 @@ bool make_cell_maps(zo_ctx* c) {
   return ok;
 }
 
-template <int MT, int BN, int STAGES, int ACC, int MODE, int CG>
+template <int MT, int BN, int STAGES, int ACC, int MODE, int CG, int XP = 0, int GB = 0>
 static cudaError_t launch_cfg(const CUtensorMap& A0, const CUtensorMap& A1, const CUtensorMap& Wm,
                               CellArgs a, int P, int sms, cudaStream_t st) {
   using C = TcCfg<MT, BN, STAGES, ACC, CG>;
-  auto kern = cell_tc_kernel<MT, BN, STAGES, ACC, MODE, CG>;
+  auto kern = cell_tc_kernel<MT, BN, STAGES, ACC, MODE, CG, XP, GB>;
   a.m_tiles = (a.B + C::ROWS - 1) / C::ROWS;
   a.n_tiles = MODE != 1 ? a.H / C::U : 1;
   a.tiles = (int64_t)P * a.m_tiles * a.n_tiles;
@@ -1009,6 +1117,16 @@ cudaError_t launch_cell_tc(const zo_ctx* ctx, int layer, int t, int B, int nprob
   a.gstride = H;
   // 256 batch rows x 256 gate rows per tile on a CTA pair, two accumulators
   // of 256 TMEM columns per CTA, six 32 KB stages
+  a.wsh = ctx->shadow + ctx->seg.off[ctx->seg.W[layer]];
+  if (ctx->cell_variant == ZO_CELL_EXACT_EPS) {
+    if (tab) return launch_cfg<1, 256, 6, 2, 2, 2, 1>(A0, A1, m.w[layer], a, P, ctx->sm_count, st);
+    return launch_cfg<1, 256, 6, 2, 0, 2, 1>(A0, A1, m.w[layer], a, P, ctx->sm_count, st);
+  }
+  if (ctx->cell_variant == ZO_CELL_DIRECT_W) {
+    if (tab)
+      return launch_cfg<1, 256, 6, 2, 2, 2, 0, 1>(A0, A1, m.w[layer], a, P, ctx->sm_count, st);
+    return launch_cfg<1, 256, 6, 2, 0, 2, 0, 1>(A0, A1, m.w[layer], a, P, ctx->sm_count, st);
+  }
   if (tab) return launch_cfg<1, 256, 6, 2, 2, 2>(A0, A1, m.w[layer], a, P, ctx->sm_count, st);
   return launch_cfg<1, 256, 6, 2, 0, 2>(A0, A1, m.w[layer], a, P, ctx->sm_count, st);
 }
@@ -1104,6 +1222,11 @@ cudaError_t launch_vocab_table(const zo_ctx* ctx, int nprobe, int probe0, uint64
   a.rowloss = nullptr;
   a.gstride = H;
   const CellMaps& m = *ctx->maps;
+  a.wsh = ctx->shadow + ctx->seg.off[ctx->seg.W[0]];
+  if (ctx->cell_variant == ZO_CELL_EXACT_EPS)
+    return launch_cfg<1, 256, 6, 2, 3, 2, 1>(m.x, m.x, m.w[0], a, P, ctx->sm_count, st);
+  if (ctx->cell_variant == ZO_CELL_DIRECT_W)
+    return launch_cfg<1, 256, 6, 2, 3, 2, 0, 1>(m.x, m.x, m.w[0], a, P, ctx->sm_count, st);
   return launch_cfg<1, 256, 6, 2, 3, 2>(m.x, m.x, m.w[0], a, P, ctx->sm_count, st);
 }
 

@@ -28,10 +28,13 @@ struct SmallArgs {
   int64_t part_blk0[kMaxSeg + 1];  // first 128-block index of each part (cumulative)
 };
 
+// One warp per 128-element block: every lane derives the block's sign words,
+// lane l handles elements l, l + 32, l + 64 and l + 96 (coalesced rows).
 __global__ void perturb_small_kernel(const SmallArgs a) {
+  const int lane = threadIdx.x & 31;
   const int64_t total = a.blocks_per_probe * a.nprobe;
-  for (int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; t < total;
-       t += (int64_t)gridDim.x * blockDim.x) {
+  const int64_t warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  for (int64_t t = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5; t < total; t += warps) {
     const int ci = (int)(t / a.blocks_per_probe);
     int64_t rb = t - (int64_t)ci * a.blocks_per_probe;
     int part = 0;
@@ -42,11 +45,15 @@ __global__ void perturb_small_kernel(const SmallArgs a) {
     const uint4 w = sign_block(a.seed, (uint32_t)(a.probe0 + ci), (uint64_t)(j0 >> 7));
     float* op = a.out + (int64_t)(2 * ci) * a.stride + a.dst[part] + kb * 128;
     float* om = op + a.stride;
-    for (int e = 0; e < n; ++e) {
-      const float th = a.theta[j0 + e];
-      const float d = sign_bit(w, j0 + e) ? -a.eps : a.eps;
-      op[e] = th + d;
-      om[e] = th - d;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int e = lane + 32 * q;
+      if (e < n) {
+        const float th = a.theta[j0 + e];
+        const float d = sign_bit(w, j0 + e) ? -a.eps : a.eps;
+        op[e] = th + d;
+        om[e] = th - d;
+      }
     }
   }
 }
@@ -83,10 +90,10 @@ cudaError_t launch_perturb_small(const zo_ctx* ctx, const float* theta, uint64_t
   a.part_blk0[np] = cum;
   a.blocks_per_probe = cum;
   a.stride = sl.stride;
-  const int64_t total = cum * nprobe;
-  int64_t grid = (total + 127) / 128;
-  if (grid > 65535) grid = 65535;
-  perturb_small_kernel<<<(int)grid, 128, 0, st>>>(a);
+  const int64_t total = cum * nprobe;       // one warp per block, 8 warps per CTA
+  int64_t grid = (total + 7) / 8;
+  if (grid > 16 * (int64_t)ctx->sm_count) grid = 16 * (int64_t)ctx->sm_count;
+  perturb_small_kernel<<<(int)grid, 256, 0, st>>>(a);
   count_launch();
   return cudaGetLastError();
 }

@@ -10,7 +10,7 @@
 #include <atomic>
 #include <vector>
 
-#include "../../include/zo.h"
+#include "../../include/zo_debug.h"
 
 namespace zo {
 
@@ -70,6 +70,8 @@ struct zo_ctx {
   // embeddings): vt[ps][v][4H] = E'_ps[v] (W_0x +- eps P)^T, built once per chunk
   float* vt = nullptr;
   bool vocab = false;
+  // how the cell GEMMs form the perturbed operand (ZO_CELL_*, include/zo_debug.h)
+  int cell_variant = 0;
   // both paths
   float* rowloss = nullptr;      // [2*chunk][B]
   // zo_step_host staging (device)
