@@ -5,6 +5,12 @@ TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
 ``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import it.
 The CUDA library never calls it, and it shares no code with the library.
 
+Two independent implementations of the same method live in this package: the
+plain C++17 one (``zo_oracle_cpu.cpp`` via ``native.py``), which the
+full-size GPU parity gates and the timed CPU baseline use, and this numpy one,
+written separately, which pins the C++ one (the two must agree to rounding)
+and serves the small GPU parity cases and the estimator-algebra pins.
+
 Sources ("Scaling Recurrent Neural Networks to a Billion Parameters with
 Zero-Order Optimization", Chaubard & Kochenderfer, arXiv 2505.17852):
 
