@@ -468,6 +468,13 @@ def main():
            "config": config,
            "roofline": roofline_for(cfg, r["kinds"], r["clocks"], pk, args.steps,
                                     probe_slice(cfg.n_pert, 0, world)[1])}
+    if cfg.dtype == "bf16":
+        # the whole step against the same peak: the plain dense forward's flops
+        # (2 n_pert B T tokens, 2 flop per multiply-add) over the step time
+        fl_step = 2.0 * forward_macs_per_token(cfg) * tokens_per_step
+        out["roofline"]["whole_step_tflops"] = round(fl_step / (r["ms"] / args.steps / 1e3) / 1e12, 2)
+        out["roofline"]["whole_step_frac"] = round(out["roofline"]["whole_step_tflops"] /
+                                                   out["roofline"]["peak"], 4)
     nu, msu, _, byu = r["kinds"]["update"]
     if nu:
         gbs = byu / (msu / 1e3) / 1e9
