@@ -38,7 +38,8 @@ import numpy as np  # noqa: E402
 import workloads as W  # noqa: E402
 
 METRIC = "CD-RGE steps/s and perturbed-forward tokens/s on 1 B200; % of roofline"
-CELL_VARIANTS = {"perturbed-operand": 0, "exact-eps": 1, "direct-w": 2}
+CELL_VARIANTS = {"single": 0, "single-exact-eps": 1, "pair": 2, "pair-exact-eps": 3,
+                 "pair-direct-w": 4}
 L2_BYTES = 126 * 1024 * 1024
 CLOCK_QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
                "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -162,7 +163,7 @@ def run_ours(args, cfg):
     coef = torch.empty(n, device=dev)
     flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
     ctx = zo.Context.for_config(cfg)
-    if args.cell_variant != "perturbed-operand":
+    if args.cell_variant != "single":
         zo.zo_debug_cell_variant(ctx, CELL_VARIANTS[args.cell_variant])
     st = torch.cuda.current_stream()
 
@@ -420,11 +421,11 @@ def main():
                     help="probes per pass (default: the workload's); smaller chunks hold less "
                          "workspace, e.g. for a profiler capture")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--cell-variant", default="perturbed-operand", choices=sorted(CELL_VARIANTS),
-                    help="how the cell GEMMs form W +- eps P (include/zo_debug.h): the bf16 tile "
-                         "perturbed in shared memory after a TMA load (default), the separate "
-                         "+-eps P product (exact eps, twice the MMA work), or the tile read into "
-                         "registers and perturbed there")
+    ap.add_argument("--cell-variant", default="single", choices=sorted(CELL_VARIANTS),
+                    help="how and on which tiles the cell GEMMs form W +- eps P "
+                         "(include/zo_debug.h): single-CTA tiles with the bf16 tile perturbed in "
+                         "shared memory (default), the separate +-eps P product (exact eps, twice "
+                         "the MMA work), CTA-pair tiles, or pair tiles with W read into registers")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -443,7 +444,7 @@ def main():
                               if world > 1 else "single GPU"),
               "l2": "flushed (256 MB write) before every timed step, flush untimed",
               "tokens": "seeded synthetic (workloads module)"}
-    if args.cell_variant != "perturbed-operand":
+    if args.cell_variant != "single":
         config["cell_variant"] = args.cell_variant
     dtype = "bf16" if cfg.dtype == "bf16" else "f32"
 

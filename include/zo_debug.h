@@ -41,26 +41,35 @@ ZO_API int zo_debug_cell_stall(zo_ctx* ctx, int32_t kind, uint64_t wait_ns, void
 
 /*
  * zo_debug_cell_variant selects, for the ZO_DTYPE_BF16 context's later calls,
- * how the tensor-core cell GEMMs apply the perturbation (the weights at
- * Theta +- eps p_i: alex-wiki "Method"; pith.science review, "What carries
- * the argument").  Every variant computes the same forward; they differ in
- * rounding and speed:
- *   ZO_CELL_PERTURBED_OPERAND (0, default)  B = bf16(bf16(W) +- bf16(eps) p),
- *       the bf16 tile of W staged in shared memory by TMA and perturbed there;
- *   ZO_CELL_EXACT_EPS (1)  G = A bf16(W)^T + A (+-bf16(eps) p)^T, the two
- *       products accumulated in fp32: the perturbation is not lost in the
- *       rounding of bf16(W) +- eps; twice the MMA work;
- *   ZO_CELL_DIRECT_W (2)  B as in 0, but the generator warps read the bf16
- *       rows of W from global memory into registers and store the perturbed
- *       tile into shared memory themselves (one shared-memory pass instead of
- *       three).
+ * how the tensor-core cell GEMMs form the weights at Theta +- eps p_i
+ * (alex-wiki "Method"; pith.science review, "What carries the argument") and
+ * on which tile form they run.  Every variant computes the same forward; they
+ * differ in rounding and speed.  Operand forms:
+ *   perturbed operand  B = bf16(bf16(W) +- bf16(eps) p), the bf16 tile of W
+ *                      staged in shared memory by TMA and perturbed there;
+ *   exact eps          G = A bf16(W)^T + A (+-bf16(eps) p)^T, the two products
+ *                      accumulated in fp32: the perturbation is not lost in
+ *                      the rounding of bf16(W) +- eps; twice the MMA work;
+ *   direct W           as the perturbed operand, but the generator warps read
+ *                      the bf16 rows of W from global memory into registers
+ *                      and store the perturbed tile themselves.
+ * Tile forms: single CTA (256 batch rows as two M = 128 MMAs per K slice on
+ * one B, one accumulator) or CTA pair (tcgen05.mma.cta_group::2, M = 256, two
+ * accumulators, each CTA loading and perturbing half of B).
+ *   ZO_CELL_SINGLE (0, default)  perturbed operand, single CTA
+ *   ZO_CELL_SINGLE_EXACT_EPS (1) exact eps, single CTA
+ *   ZO_CELL_PAIR (2)             perturbed operand, CTA pair
+ *   ZO_CELL_PAIR_EXACT_EPS (3)   exact eps, CTA pair
+ *   ZO_CELL_PAIR_DIRECT_W (4)    direct W, CTA pair
  * Embedding rows and biases are perturbed in fp32 in every variant.  Returns
  * ZO_ERR_UNSUPPORTED for ZO_DTYPE_FP32 contexts, ZO_ERR_INVALID_ARG for an
  * unknown variant.  Synchronous, host only.
  */
-#define ZO_CELL_PERTURBED_OPERAND 0
-#define ZO_CELL_EXACT_EPS 1
-#define ZO_CELL_DIRECT_W 2
+#define ZO_CELL_SINGLE 0
+#define ZO_CELL_SINGLE_EXACT_EPS 1
+#define ZO_CELL_PAIR 2
+#define ZO_CELL_PAIR_EXACT_EPS 3
+#define ZO_CELL_PAIR_DIRECT_W 4
 ZO_API int zo_debug_cell_variant(zo_ctx* ctx, int32_t variant);
 
 ZO_API int zo_debug_cell_preact(zo_ctx* ctx, const float* theta_dev, uint64_t step_seed,

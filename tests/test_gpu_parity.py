@@ -356,7 +356,8 @@ def _bf16(x):
 
 
 @pytest.mark.parametrize("B,E,H", [(200, 64, 64), (128, 128, 128), (300, 256, 1024)])
-@pytest.mark.parametrize("xp", [0, 1, 2], ids=["perturbed_operand", "exact_eps", "direct_w"])
+@pytest.mark.parametrize("xp", [0, 1, 2, 3, 4], ids=["single", "single_exact_eps", "pair",
+                                                    "pair_exact_eps", "pair_direct_w"])
 def test_tc_cell_preactivation_matches_emulation(B, E, H, xp):
     """One tensor-core cell step (layer 0, t = 0) against an fp64 evaluation of
     the same bf16 operands: x = bf16(E +- eps p) and either
@@ -383,7 +384,7 @@ def test_tc_cell_preactivation_matches_emulation(B, E, H, xp):
         pb = O.probe_signs(seed, i, offb, 4 * H).astype(np.float32)
         for s, sg in ((0, 1.0), (1, -1.0)):
             x = _bf16((theta[offE:offE + V * E].reshape(V, E) + np.float32(sg) * eps * pE)[tok[:, 0]])
-            if xp == 1:
+            if xp in (zo.ZO_CELL_SINGLE_EXACT_EPS, zo.ZO_CELL_PAIR_EXACT_EPS):
                 Wp = _bf16(Wt).astype(np.float64) + \
                     float(sg) * float(_bf16(np.float32(eps))) * pW.astype(np.float64)
             else:
@@ -396,7 +397,8 @@ def test_tc_cell_preactivation_matches_emulation(B, E, H, xp):
                 (i, s, float(err.max()))
 
 
-@pytest.mark.parametrize("xp", [0, 1, 2], ids=["perturbed_operand", "exact_eps", "direct_w"])
+@pytest.mark.parametrize("xp", [0, 1, 2, 3, 4], ids=["single", "single_exact_eps", "pair",
+                                                    "pair_exact_eps", "pair_direct_w"])
 @pytest.mark.parametrize("V,E,H,L,B,T,n", [(50, 64, 64, 2, 200, 4, 4), (50, 128, 256, 1, 128, 3, 3),
                                            (50, 512, 64, 2, 256, 3, 2)])
 def test_bf16_small_matches_oracle(V, E, H, L, B, T, n, xp):

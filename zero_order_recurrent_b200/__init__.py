@@ -35,7 +35,8 @@ EXPORTS = (
     "zo_probe_losses_slice", "zo_loss", "zo_coeffs_forward", "zo_debug_cell_stall",
     "zo_debug_cell_variant",
 )
-ZO_CELL_PERTURBED_OPERAND, ZO_CELL_EXACT_EPS, ZO_CELL_DIRECT_W = 0, 1, 2
+ZO_CELL_SINGLE, ZO_CELL_SINGLE_EXACT_EPS, ZO_CELL_PAIR, ZO_CELL_PAIR_EXACT_EPS, \
+    ZO_CELL_PAIR_DIRECT_W = 0, 1, 2, 3, 4
 ZO_STATIC_SCRATCH_FLOATS = 65536
 ZO_MAX_UPDATE_PROBES = 8192
 ZO_KIND_CELL, ZO_KIND_LOSS, ZO_KIND_UPDATE, ZO_KIND_OTHER = 0, 1, 2, 3

@@ -41,9 +41,10 @@
 
 namespace zo {
 
-constexpr int kTcThreads = 448;
-constexpr int kGenThreads = 256;
-constexpr int kGenWarps = kGenThreads / 32;
+// generator warps: eight on single-CTA tiles (256 W rows per stage, one row a
+// thread), four on pair tiles (128 rows, still one row a thread)
+__host__ __device__ constexpr int gen_warps(int cg) { return cg == 2 ? 4 : 8; }
+__host__ __device__ constexpr int tc_threads(int cg) { return (2 + gen_warps(cg) + 4) * 32; }
 constexpr uint64_t kWaitLimitNs = kDefaultWaitNs;   // default bound of a wait
 
 struct CellArgs {
@@ -113,11 +114,22 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Memory scope of the pair's cross-CTA barrier traffic: 1 = release/acquire
+// at cluster scope; 0 = the default (CTA-scope) forms of arrive and wait on
+// the remote barrier.
+#ifndef ZO_PAIR_SYNC_CLUSTER
+#define ZO_PAIR_SYNC_CLUSTER 1
+#endif
+
 __device__ __forceinline__ bool mbar_try_cluster(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
+#if ZO_PAIR_SYNC_CLUSTER
       "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+#else
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+#endif
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
       : "r"(bar), "r"(parity)
@@ -248,11 +260,15 @@ __device__ __forceinline__ uint32_t peer_addr(uint32_t addr, uint32_t rank) {
   return r;
 }
 
-// arrive on a barrier of the cluster (here: CTA 0's), releasing this thread's
-// earlier writes at cluster scope
+
+// arrive on a barrier of the cluster (here: CTA 0's)
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+#if ZO_PAIR_SYNC_CLUSTER
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
                : "memory");
+#else
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+#endif
 }
 
 __device__ __forceinline__ void cluster_sync_all() {
@@ -384,11 +400,13 @@ struct TcCfg {
 // only A arrives by TMA.  The W tile then crosses shared memory once (the
 // store) instead of three times (TMA write, load, store).
 template <int MT, int BN, int STAGES, int ACC, int MODE, int CG, int XP = 0, int GB = 0>
-__global__ void __launch_bounds__(kTcThreads, 1)
+__global__ void __launch_bounds__(tc_threads(CG), 1)
     cell_tc_kernel(const __grid_constant__ CUtensorMap mapA0, const __grid_constant__ CUtensorMap mapA1,
                    const __grid_constant__ CUtensorMap mapW, const CellArgs a, int P) {
   using C = TcCfg<MT, BN, STAGES, ACC, CG>;
   constexpr bool PAIR = CG == 2;
+  constexpr int kGenWarps = gen_warps(CG);
+  constexpr int kGenThreads = kGenWarps * 32;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -425,7 +443,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(full_bar(s), 1);
-      mbar_init(ready_bar(s), kGenWarps * CG);
+      // CTA 1's generator warps arrive on their own barrier; one thread of
+      // CTA 1 forwards a single arrival per stage to CTA 0's
+      mbar_init(ready_bar(s), kGenWarps + (PAIR && rank == 0 ? 1 : 0));
       mbar_init(empty_bar(s), 1);
     }
     for (int b = 0; b < ACC; ++b) {
@@ -515,6 +535,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    if (PAIR && lane == 0 && rank == 1) {
+      // forwarder: once this CTA's generator warps have released a stage
+      // (CTA-scope arrivals on its own barrier), pass one cluster-scope
+      // arrival to CTA 0, whose MMA thread reads this CTA's half of the stage
+      uint32_t it = 0;
+      bool ok = true;
+      for (int64_t tile = walker; tile < a.tiles && ok; tile += walkers) {
+        for (int kb = a.kbeg; kb < kend; ++kb, ++it) {
+          const int s = it % STAGES;
+          if (!mbar_wait(ready_bar(s), (it / STAGES) & 1, abort_flag, a.err, a.wait_ns)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_cluster(peer_addr(ready_bar(s), 0));
+        }
+      }
+    }
     if (lane == 0 && rank == 0) {
       constexpr uint32_t idesc = umma_idesc(128 * CG, BN);
       uint32_t it = 0, tcount = 0;
@@ -588,24 +625,36 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     uint32_t it = 0;
     bool ok = true;
     if constexpr (GB) {
-      // this thread: row r = gt of the CTA's B half, chunks c0 .. c0 + 3 (64
-      // contiguous bytes of the row's 128-byte K slice)
-      static_assert(PAIR && XP == 0 && RPT == 1 && CPT == 4, "direct W loads: pair tiles");
+      // Coalesced rows: warp w owns rows w*WR .. w*WR + WR - 1 of the CTA's B
+      // half; lane l reads the 16-byte chunk c = l & 7 of rows
+      // w*WR + 4 i + (l >> 3), i < WR/4, so eight lanes cover a row's 128 bytes.
+      // Lane l (l < WR) derives the Philox block of row w*WR + l and hands
+      // the two words a row's 64 elements need to the lanes that use them.
+      static_assert(PAIR && XP == 0, "direct W loads: pair tiles");
       constexpr int D = 3;                           // stages of loads in flight
-      const int r = gt;
-      const int g = (int)rank * C::GPC + r / C::U, u = r % C::U;
-      const int64_t Rbase = (int64_t)g * a.gstride + u;
-      uint4 buf[D][CPT];
-      // load cursor: (tile, K stage) of the next loads, D stages ahead
+      constexpr int WR = BL / kGenWarps;             // rows per warp
+      constexpr int NI = WR / 4;                     // rows per lane
+      const int gw = (threadIdx.x - 64) >> 5;        // generator warp 0..7
+      const int c = lane & 7, rs = lane >> 3;
+      const int rp = gw * WR + (lane % WR);          // the row whose Philox block this lane derives
+      const int gp = (int)rank * C::GPC + rp / C::U, up = rp % C::U;
+      int64_t rbase[NI];
+#pragma unroll
+      for (int i = 0; i < NI; ++i) {
+        const int r = gw * WR + 4 * i + rs;
+        const int g = (int)rank * C::GPC + r / C::U, u = r % C::U;
+        rbase[i] = (int64_t)g * a.gstride + u;
+      }
+      uint4 buf[D][NI];
       int64_t ltile = walker;
       int lkb = a.kbeg;
-      auto issue = [&](uint4 (&dst)[CPT]) {
+      auto issue = [&](uint4 (&dst)[NI]) {
         if (ltile < a.tiles) {
           const TileCoord lt = decode_tile(a, ltile, P);
-          const uint4* src = reinterpret_cast<const uint4*>(
-              a.wsh + (Rbase + (int64_t)lt.n * C::U) * a.Ktot + (int64_t)lkb * 64 + c0 * 8);
 #pragma unroll
-          for (int cc = 0; cc < CPT; ++cc) dst[cc] = __ldg(src + cc);
+          for (int i = 0; i < NI; ++i)
+            dst[i] = __ldg(reinterpret_cast<const uint4*>(
+                a.wsh + (rbase[i] + (int64_t)lt.n * C::U) * a.Ktot + (int64_t)lkb * 64 + c * 8));
           if (++lkb == a.nk) {
             lkb = a.kbeg;
             ltile += walkers;
@@ -630,30 +679,33 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             } else {
               const uint32_t probe = (uint32_t)(a.probe0 + (ct.ps >> 1));
               const uint32_t e2 = (ct.ps & 1) ? epsn2 : epsp2;
-              const int64_t R = Rbase + (int64_t)ct.n * C::U;
-              const int64_t j0 = a.offW + R * a.Ktot + (int64_t)ckb * 64;
-              const int64_t q = j0 >> 7;
+              // this lane's Philox row: words of the stage's half-block
+              const int64_t jp = a.offW + ((int64_t)gp * a.gstride + (int64_t)ct.n * C::U + up) *
+                                              a.Ktot + (int64_t)ckb * 64;
+              const int64_t q = jp >> 7;
               if (q != cq) {
                 cw = sign_block(a.seed, probe, (uint64_t)q);
                 cq = q;
               }
-              const bool upper = (j0 >> 6) & 1;
-              const uint32_t wsel = c0 < 4 ? (upper ? cw.z : cw.x) : (upper ? cw.w : cw.y);
-              uint8_t* row = smem + s * C::STAGE + C::A_BYTES + r * 128;
+              const bool upper = (jp >> 6) & 1;
+              const uint32_t wlo = upper ? cw.z : cw.x, whi = upper ? cw.w : cw.y;
+              uint8_t* tileB = smem + s * C::STAGE + C::A_BYTES;
 #pragma unroll
-              for (int cc = 0; cc < CPT; ++cc) {
-                const int c16 = c0 + cc;
-                const uint32_t w = wsel >> (4 * (c16 & 3));
-                uint4 v = buf[d][cc];
+              for (int i = 0; i < NI; ++i) {
+                const int r = gw * WR + 4 * i + rs;
+                const uint32_t lo = __shfl_sync(0xffffffffu, wlo, 4 * i + rs);
+                const uint32_t hi = __shfl_sync(0xffffffffu, whi, 4 * i + rs);
+                const uint32_t w = (c < 4 ? lo : hi) >> (4 * (c & 3));
+                uint4 v = buf[d][i];
                 v.x = bf16x2_add(v.x, ((w << 15) & 0x80008000u) ^ e2);
                 v.y = bf16x2_add(v.y, ((w << 14) & 0x80008000u) ^ e2);
                 v.z = bf16x2_add(v.z, ((w << 13) & 0x80008000u) ^ e2);
                 v.w = bf16x2_add(v.w, ((w << 12) & 0x80008000u) ^ e2);
-                *reinterpret_cast<uint4*>(row + ((c16 ^ (r & 7)) << 4)) = v;
+                *reinterpret_cast<uint4*>(tileB + r * 128 + ((c ^ (r & 7)) << 4)) = v;
               }
               fence_async_smem();
               __syncwarp();
-              if (lane == 0) report(ready_bar(s));
+              if (lane == 0) mbar_arrive(ready_bar(s));
               issue(buf[d]);
               ++it;
               if (++ckb == a.nk) {
@@ -724,7 +776,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         fence_async_smem();
         __syncwarp();
-        if (lane == 0) report(ready_bar(s));
+        if (lane == 0) mbar_arrive(ready_bar(s));
       }
     }
   } else {
@@ -1033,7 +1085,7 @@ static cudaError_t launch_cfg(const CUtensorMap& A0, const CUtensorMap& A1, cons
   if (e != cudaSuccess) return e;
   if constexpr (CG == 1) {
     const int64_t grid = a.tiles < sms ? a.tiles : sms;
-    kern<<<(int)grid, kTcThreads, C::SMEM, st>>>(A0, A1, Wm, a, P);
+    kern<<<(int)grid, tc_threads(CG), C::SMEM, st>>>(A0, A1, Wm, a, P);
     count_launch();
     return cudaGetLastError();
   } else {
@@ -1045,7 +1097,7 @@ static cudaError_t launch_cfg(const CUtensorMap& A0, const CUtensorMap& A1, cons
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
-    cfg.blockDim = dim3(kTcThreads, 1, 1);
+    cfg.blockDim = dim3(tc_threads(CG), 1, 1);
     cfg.dynamicSmemBytes = C::SMEM;
     cfg.stream = st;
     cfg.attrs = attr;
@@ -1118,17 +1170,27 @@ cudaError_t launch_cell_tc(const zo_ctx* ctx, int layer, int t, int B, int nprob
   // 256 batch rows x 256 gate rows per tile on a CTA pair, two accumulators
   // of 256 TMEM columns per CTA, six 32 KB stages
   a.wsh = ctx->shadow + ctx->seg.off[ctx->seg.W[layer]];
-  if (ctx->cell_variant == ZO_CELL_EXACT_EPS) {
-    if (tab) return launch_cfg<1, 256, 6, 2, 2, 2, 1>(A0, A1, m.w[layer], a, P, ctx->sm_count, st);
-    return launch_cfg<1, 256, 6, 2, 0, 2, 1>(A0, A1, m.w[layer], a, P, ctx->sm_count, st);
+  const int sms = ctx->sm_count;
+  const CUtensorMap& Wm = m.w[layer];
+  switch (ctx->cell_variant) {
+    case ZO_CELL_SINGLE_EXACT_EPS:
+      if (tab) return launch_cfg<2, 256, 3, 1, 2, 1, 1>(A0, A1, Wm, a, P, sms, st);
+      return launch_cfg<2, 256, 3, 1, 0, 1, 1>(A0, A1, Wm, a, P, sms, st);
+    case ZO_CELL_PAIR:
+      if (tab) return launch_cfg<1, 256, 6, 2, 2, 2>(A0, A1, Wm, a, P, sms, st);
+      return launch_cfg<1, 256, 6, 2, 0, 2>(A0, A1, Wm, a, P, sms, st);
+    case ZO_CELL_PAIR_EXACT_EPS:
+      if (tab) return launch_cfg<1, 256, 6, 2, 2, 2, 1>(A0, A1, Wm, a, P, sms, st);
+      return launch_cfg<1, 256, 6, 2, 0, 2, 1>(A0, A1, Wm, a, P, sms, st);
+    case ZO_CELL_PAIR_DIRECT_W:
+      if (tab) return launch_cfg<1, 256, 6, 2, 2, 2, 0, 1>(A0, A1, Wm, a, P, sms, st);
+      return launch_cfg<1, 256, 6, 2, 0, 2, 0, 1>(A0, A1, Wm, a, P, sms, st);
+    default:
+      // one CTA per 256 x 256 tile: two M = 128 MMAs per K slice on one B,
+      // one accumulator, three 64 KB stages
+      if (tab) return launch_cfg<2, 256, 3, 1, 2, 1>(A0, A1, Wm, a, P, sms, st);
+      return launch_cfg<2, 256, 3, 1, 0, 1>(A0, A1, Wm, a, P, sms, st);
   }
-  if (ctx->cell_variant == ZO_CELL_DIRECT_W) {
-    if (tab)
-      return launch_cfg<1, 256, 6, 2, 2, 2, 0, 1>(A0, A1, m.w[layer], a, P, ctx->sm_count, st);
-    return launch_cfg<1, 256, 6, 2, 0, 2, 0, 1>(A0, A1, m.w[layer], a, P, ctx->sm_count, st);
-  }
-  if (tab) return launch_cfg<1, 256, 6, 2, 2, 2>(A0, A1, m.w[layer], a, P, ctx->sm_count, st);
-  return launch_cfg<1, 256, 6, 2, 0, 2>(A0, A1, m.w[layer], a, P, ctx->sm_count, st);
 }
 
 // Output projection + softmax cross-entropy for step t on the same
@@ -1223,11 +1285,19 @@ cudaError_t launch_vocab_table(const zo_ctx* ctx, int nprobe, int probe0, uint64
   a.gstride = H;
   const CellMaps& m = *ctx->maps;
   a.wsh = ctx->shadow + ctx->seg.off[ctx->seg.W[0]];
-  if (ctx->cell_variant == ZO_CELL_EXACT_EPS)
-    return launch_cfg<1, 256, 6, 2, 3, 2, 1>(m.x, m.x, m.w[0], a, P, ctx->sm_count, st);
-  if (ctx->cell_variant == ZO_CELL_DIRECT_W)
-    return launch_cfg<1, 256, 6, 2, 3, 2, 0, 1>(m.x, m.x, m.w[0], a, P, ctx->sm_count, st);
-  return launch_cfg<1, 256, 6, 2, 3, 2>(m.x, m.x, m.w[0], a, P, ctx->sm_count, st);
+  const int sms = ctx->sm_count;
+  switch (ctx->cell_variant) {
+    case ZO_CELL_SINGLE_EXACT_EPS:
+      return launch_cfg<2, 256, 3, 1, 3, 1, 1>(m.x, m.x, m.w[0], a, P, sms, st);
+    case ZO_CELL_PAIR:
+      return launch_cfg<1, 256, 6, 2, 3, 2>(m.x, m.x, m.w[0], a, P, sms, st);
+    case ZO_CELL_PAIR_EXACT_EPS:
+      return launch_cfg<1, 256, 6, 2, 3, 2, 1>(m.x, m.x, m.w[0], a, P, sms, st);
+    case ZO_CELL_PAIR_DIRECT_W:
+      return launch_cfg<1, 256, 6, 2, 3, 2, 0, 1>(m.x, m.x, m.w[0], a, P, sms, st);
+    default:
+      return launch_cfg<2, 256, 3, 1, 3, 1>(m.x, m.x, m.w[0], a, P, sms, st);
+  }
 }
 
 }  // namespace zo

@@ -359,7 +359,7 @@ static int probe_losses_range(zo_ctx* ctx, const float* theta, uint64_t seed, in
     const bool vocab = ctx->vocab;
     if (vocab) {
       // executed flops: the 256-row tile over the vocabulary rows
-      const double fl = 2.0 * P * 256.0 * Ee * 4.0 * Hh * (ctx->cell_variant == ZO_CELL_EXACT_EPS ? 2.0 : 1.0);
+      const double fl = 2.0 * P * 256.0 * Ee * 4.0 * Hh * ((ctx->cell_variant == ZO_CELL_SINGLE_EXACT_EPS || ctx->cell_variant == ZO_CELL_PAIR_EXACT_EPS) ? 2.0 : 1.0);
       ZO_CUDA(timed(ctx, st, ZO_KIND_OTHER, 0.0, 0.0, [&] { return launch_vocab_x(ctx, np, st); }));
       ZO_CUDA(timed(ctx, st, ZO_KIND_CELL, fl, 0.0, [&] {
         return launch_vocab_table(ctx, np, probe_begin + p0, seed, eps, st);
@@ -378,7 +378,7 @@ static int probe_losses_range(zo_ctx* ctx, const float* theta, uint64_t seed, in
         const double Kin = (vocab && l == 0) ? 0.0 : (double)(l == 0 ? Ee : Hh);
         const double Krun = Kin + (t == 0 ? 0.0 : (double)Hh);
         // executed flops (twice over with the separate +-eps P product)
-        const double fl = 2.0 * P * B * Krun * 4.0 * Hh * (ctx->cell_variant == ZO_CELL_EXACT_EPS ? 2.0 : 1.0);
+        const double fl = 2.0 * P * B * Krun * 4.0 * Hh * ((ctx->cell_variant == ZO_CELL_SINGLE_EXACT_EPS || ctx->cell_variant == ZO_CELL_PAIR_EXACT_EPS) ? 2.0 : 1.0);
         ZO_CUDA(timed(ctx, st, ZO_KIND_CELL, fl, 0.0, [&] {
           return launch_cell_tc(ctx, l, t, B, np, probe_begin + p0, seed, eps, nullptr, tokens, T,
                                 vocab, st);
@@ -552,7 +552,7 @@ int zo_profile_read(zo_ctx* ctx, int32_t kind, int64_t* launches, double* total_
 }
 
 int zo_debug_cell_variant(zo_ctx* ctx, int32_t variant) {
-  if (!ctx || variant < ZO_CELL_PERTURBED_OPERAND || variant > ZO_CELL_DIRECT_W)
+  if (!ctx || variant < ZO_CELL_SINGLE || variant > ZO_CELL_PAIR_DIRECT_W)
     return ZO_ERR_INVALID_ARG;
   if (ctx->spec.dtype != ZO_DTYPE_BF16) return ZO_ERR_UNSUPPORTED;
   ctx->cell_variant = variant;
