@@ -312,13 +312,15 @@ def roofline_for(cfg, kinds, clocks, pk, steps, n_rank):
 class OracleSampler:
     """The C++ fp64 oracle (as it stands) on bounded samples of one CD-RGE step
     of `cfg`, on this host's cores.  A sample is one probe (both signs) over
-    R batch rows plus the update of a contiguous run of m parameters with all
-    n_pert probes; a full step extrapolates linearly:
-        t_step = t_forward(R rows, 2 forwards) x n_pert x B / R + t_update(m) x d_pad / m.
-    R is the largest row count (<= 32, <= B) whose sample fits `target_s`,
-    found from a one-row calibration forward."""
+    R2 = min(B, 8) batch rows plus the update of a contiguous run of m
+    parameters with all n_pert probes.  The oracle's time for one probe grows
+    linearly in the rows it evaluates, t(r) = t(1) + (r - 1) s, with an
+    intercept that does not shrink with rows (it rebuilds every perturbed
+    weight at every step), so one probe at 1 row and at R2 rows fix the line,
+    and a full step is extrapolated as
+        t_step = n_pert t(B) + t_update(m) d_pad / m."""
 
-    def __init__(self, cfg, target_s, rank=0):
+    def __init__(self, cfg, rank=0):
         from oracle import native
         self.cfg = cfg
         self.N = native.Oracle()
@@ -329,13 +331,14 @@ class OracleSampler:
         self.d_pad = int(self.theta.size)
         self.m = min(self.d_pad, 1 << 22)
         self.coef = np.random.default_rng(0).standard_normal(cfg.n_pert) * 1e-3
-        t0 = time.perf_counter()
-        self.N.probe_row_losses(self.theta, self.spec, W.step_seed(0), [0], cfg.eps,
-                                self.tok, self.tgt, rows=[0])
-        t_row = max(time.perf_counter() - t0, 1e-6)      # one forward, one row
-        self.calib_s = t_row
-        self.R = int(max(1, min(cfg.batch, 32, target_s / (2.0 * t_row))))
-        self.rows = np.arange(self.R)
+        self.R2 = min(cfg.batch, 8)
+        self.rows = np.arange(self.R2)
+        self.t1 = None
+        if cfg.batch > 1:
+            t0 = time.perf_counter()
+            self.N.probe_row_losses(self.theta, self.spec, W.step_seed(0), [0], cfg.eps,
+                                    self.tok, self.tgt, rows=[0])
+            self.t1 = time.perf_counter() - t0       # one probe, both signs, one row
 
     def sample(self, k):
         """One timed sample with probe k mod n_pert; returns (t_forward, t_update)."""
@@ -348,22 +351,34 @@ class OracleSampler:
         self.N.update_range(self.theta, self.spec, seed, cfg.n_pert, self.coef, 0, self.m)
         return t1 - t0, time.perf_counter() - t1
 
+    def probe_seconds_full_batch(self, t_fwd):
+        """One probe (both signs) over all B rows from the line through
+        (1, t1) and (R2, t_fwd)."""
+        B = self.cfg.batch
+        if self.t1 is None or self.R2 <= 1:
+            return t_fwd * B / self.R2
+        slope = max(0.0, (t_fwd - self.t1) / (self.R2 - 1))
+        return max(t_fwd, self.t1 + (B - 1) * slope)
+
     def step_seconds(self, t_fwd, t_upd):
-        cfg = self.cfg
-        return t_fwd * cfg.n_pert * cfg.batch / self.R + t_upd * self.d_pad / self.m
+        return (self.cfg.n_pert * self.probe_seconds_full_batch(t_fwd) +
+                t_upd * self.d_pad / self.m)
 
     def describe(self, n_samples):
         cfg = self.cfg
-        return (f"{n_samples} sample(s), each one probe (both signs) over {self.R} of {cfg.batch} "
+        fit = ("" if self.t1 is None or self.R2 <= 1 else
+               f"; one probe over 1 row took {self.t1:.2f} s, the line through that and the "
+               f"{self.R2}-row samples gives the {cfg.batch}-row time")
+        return (f"{n_samples} sample(s), each one probe (both signs) over {self.R2} of {cfg.batch} "
                 f"rows at T={cfg.seq} plus the update of {self.m} of {self.d_pad} parameters with "
-                f"all {cfg.n_pert} probes; extrapolated linearly to the full step "
-                f"({cfg.n_pert} probes x {cfg.batch} rows, {self.d_pad} parameters)")
+                f"all {cfg.n_pert} probes; extrapolated to the full step ({cfg.n_pert} probes x "
+                f"{cfg.batch} rows, {self.d_pad} parameters){fit}")
 
 
 def oracle_sample(cfg, budget_s=15.0, rank=0):
     """cpu_baseline: the C++ fp64 oracle timed on a bounded sample of one step."""
     t_all = time.perf_counter()
-    S = OracleSampler(cfg, target_s=0.8 * budget_s, rank=rank)
+    S = OracleSampler(cfg, rank=rank)
     t_fwd, t_upd, n = 0.0, 0.0, 0
     while n < cfg.n_pert and (n == 0 or time.perf_counter() - t_all < budget_s):
         f, u = S.sample(n)
@@ -372,7 +387,7 @@ def oracle_sample(cfg, budget_s=15.0, rank=0):
     return {"value": 1.0 / step_s, "unit": "steps/s", "cores": S.cores, "kind": "oracle",
             "impl": "C++17 fp64, std::thread (oracle/zo_oracle_cpu.cpp)",
             "sample": S.describe(n), "extrapolated": True,
-            "perturbed_tokens_per_s": 2 * n * S.R * cfg.seq / t_fwd,
+            "perturbed_tokens_per_s": 2 * n * S.R2 * cfg.seq / t_fwd,
             "seconds": round(time.perf_counter() - t_all, 2)}
 
 
@@ -380,8 +395,7 @@ def run_reference(args, cfg, config):
     """The reference arm: the C++ fp64 oracle as it stands, on this host's
     cores, W warm-up and K timed samples (each a bounded sample of one step,
     sized so the whole run stays within a few minutes), extrapolated."""
-    per = min(10.0, max(0.5, 150.0 / (args.steps + args.warmup)))
-    S = OracleSampler(cfg, target_s=per)
+    S = OracleSampler(cfg)
     for k in range(args.warmup):
         S.sample(k)
     t0 = time.perf_counter()
@@ -397,7 +411,7 @@ def run_reference(args, cfg, config):
           "impl": "C++17 fp64, std::thread (oracle/zo_oracle_cpu.cpp)",
           "sample": S.describe(args.steps), "extrapolated": True}
     return {"metric": METRIC, "impl": "reference", "value": v, "unit": "steps/s",
-            "perturbed_tokens_per_s": 2 * S.R * cfg.seq / t_fwd, "n_gpus": 1,
+            "perturbed_tokens_per_s": 2 * S.R2 * cfg.seq / t_fwd, "n_gpus": 1,
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": wall / args.steps * 1e3,
             "ms_per_full_step_extrapolated": 1e3 / v,
