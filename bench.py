@@ -39,7 +39,7 @@ import workloads as W  # noqa: E402
 
 METRIC = "CD-RGE steps/s and perturbed-forward tokens/s on 1 B200; % of roofline"
 CELL_VARIANTS = {"single": 0, "single-exact-eps": 1, "pair": 2, "pair-exact-eps": 3,
-                 "pair-direct-w": 4}
+                 "pair-direct-w": 4, "single-epi8": 5}
 L2_BYTES = 126 * 1024 * 1024
 CLOCK_QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
                "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"

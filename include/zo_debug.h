@@ -61,6 +61,10 @@ ZO_API int zo_debug_cell_stall(zo_ctx* ctx, int32_t kind, uint64_t wait_ns, void
  *   ZO_CELL_PAIR (2)             perturbed operand, CTA pair
  *   ZO_CELL_PAIR_EXACT_EPS (3)   exact eps, CTA pair
  *   ZO_CELL_PAIR_DIRECT_W (4)    direct W, CTA pair
+ *   ZO_CELL_SINGLE_EPI8 (5)      perturbed operand, single CTA, with four
+ *                                generator warps (two W rows a thread) and
+ *                                eight epilogue warps (two per TMEM lane
+ *                                quadrant, half the units each)
  * Embedding rows and biases are perturbed in fp32 in every variant.  Returns
  * ZO_ERR_UNSUPPORTED for ZO_DTYPE_FP32 contexts, ZO_ERR_INVALID_ARG for an
  * unknown variant.  Synchronous, host only.
@@ -70,6 +74,7 @@ ZO_API int zo_debug_cell_stall(zo_ctx* ctx, int32_t kind, uint64_t wait_ns, void
 #define ZO_CELL_PAIR 2
 #define ZO_CELL_PAIR_EXACT_EPS 3
 #define ZO_CELL_PAIR_DIRECT_W 4
+#define ZO_CELL_SINGLE_EPI8 5
 ZO_API int zo_debug_cell_variant(zo_ctx* ctx, int32_t variant);
 
 ZO_API int zo_debug_cell_preact(zo_ctx* ctx, const float* theta_dev, uint64_t step_seed,

@@ -356,8 +356,9 @@ def _bf16(x):
 
 
 @pytest.mark.parametrize("B,E,H", [(200, 64, 64), (128, 128, 128), (300, 256, 1024)])
-@pytest.mark.parametrize("xp", [0, 1, 2, 3, 4], ids=["single", "single_exact_eps", "pair",
-                                                    "pair_exact_eps", "pair_direct_w"])
+@pytest.mark.parametrize("xp", [0, 1, 2, 3, 4, 5], ids=["single", "single_exact_eps", "pair",
+                                                       "pair_exact_eps", "pair_direct_w",
+                                                       "single_epi8"])
 def test_tc_cell_preactivation_matches_emulation(B, E, H, xp):
     """One tensor-core cell step (layer 0, t = 0) against an fp64 evaluation of
     the same bf16 operands: x = bf16(E +- eps p) and either
@@ -397,8 +398,9 @@ def test_tc_cell_preactivation_matches_emulation(B, E, H, xp):
                 (i, s, float(err.max()))
 
 
-@pytest.mark.parametrize("xp", [0, 1, 2, 3, 4], ids=["single", "single_exact_eps", "pair",
-                                                    "pair_exact_eps", "pair_direct_w"])
+@pytest.mark.parametrize("xp", [0, 1, 2, 3, 4, 5], ids=["single", "single_exact_eps", "pair",
+                                                       "pair_exact_eps", "pair_direct_w",
+                                                       "single_epi8"])
 @pytest.mark.parametrize("V,E,H,L,B,T,n", [(50, 64, 64, 2, 200, 4, 4), (50, 128, 256, 1, 128, 3, 3),
                                            (50, 512, 64, 2, 256, 3, 2)])
 def test_bf16_small_matches_oracle(V, E, H, L, B, T, n, xp):

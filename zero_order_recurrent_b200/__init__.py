@@ -36,7 +36,7 @@ EXPORTS = (
     "zo_debug_cell_variant",
 )
 ZO_CELL_SINGLE, ZO_CELL_SINGLE_EXACT_EPS, ZO_CELL_PAIR, ZO_CELL_PAIR_EXACT_EPS, \
-    ZO_CELL_PAIR_DIRECT_W = 0, 1, 2, 3, 4
+    ZO_CELL_PAIR_DIRECT_W, ZO_CELL_SINGLE_EPI8 = 0, 1, 2, 3, 4, 5
 ZO_STATIC_SCRATCH_FLOATS = 65536
 ZO_MAX_UPDATE_PROBES = 8192
 ZO_KIND_CELL, ZO_KIND_LOSS, ZO_KIND_UPDATE, ZO_KIND_OTHER = 0, 1, 2, 3

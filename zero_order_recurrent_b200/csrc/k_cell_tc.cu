@@ -43,8 +43,14 @@ namespace zo {
 
 // generator warps: eight on single-CTA tiles (256 W rows per stage, one row a
 // thread), four on pair tiles (128 rows, still one row a thread)
-__host__ __device__ constexpr int gen_warps(int cg) { return cg == 2 ? 4 : 8; }
-__host__ __device__ constexpr int tc_threads(int cg) { return (2 + gen_warps(cg) + 4) * 32; }
+// (ew = 8 on single-CTA tiles: four generator warps, two rows a thread, and
+// eight epilogue warps, two per TMEM lane quadrant, each taking half the units)
+__host__ __device__ constexpr int gen_warps(int cg, int ew = 4) {
+  return cg == 2 ? 4 : (ew == 8 ? 4 : 8);
+}
+__host__ __device__ constexpr int tc_threads(int cg, int ew = 4) {
+  return (2 + gen_warps(cg, ew) + ew) * 32;
+}
 constexpr uint64_t kWaitLimitNs = kDefaultWaitNs;   // default bound of a wait
 
 struct CellArgs {
@@ -364,7 +370,7 @@ __device__ __forceinline__ TileCoord decode_tile(const CellArgs& a, int64_t tile
   return c;
 }
 
-template <int MT, int BN, int STAGES, int ACC, int CG>
+template <int MT, int BN, int STAGES, int ACC, int CG, int EW = 4>
 struct TcCfg {
   static constexpr int U = BN / 4;                  // hidden units per tile
   static constexpr int BL = BN / CG;                // gate rows of B held by this CTA
@@ -376,7 +382,7 @@ struct TcCfg {
   static constexpr int ROWS = 128 * MT * CG;        // batch rows per tile
   static constexpr int COLS = MT * BN;              // TMEM columns per accumulator
   static constexpr int TMEM_COLS = COLS * ACC;
-  static constexpr int EPI = 4 * 4 * U * 4;          // per epilogue warp: bias slice [4][U]
+  static constexpr int EPI = EW * 4 * U * 4;         // per epilogue warp: bias slice [4][U]
   static constexpr int SMEM = STAGES * STAGE + 1024 + 256 + EPI;
   static_assert(BN % 64 == 0 && BN <= 256, "BN");
   static_assert(CG == 1 || (CG == 2 && MT == 1 && BN == 256), "pair tiles are 256 x 256");
@@ -399,13 +405,14 @@ struct TcCfg {
 // +-eps p there and store the perturbed tile into shared memory (swizzled);
 // only A arrives by TMA.  The W tile then crosses shared memory once (the
 // store) instead of three times (TMA write, load, store).
-template <int MT, int BN, int STAGES, int ACC, int MODE, int CG, int XP = 0, int GB = 0>
-__global__ void __launch_bounds__(tc_threads(CG), 1)
+template <int MT, int BN, int STAGES, int ACC, int MODE, int CG, int XP = 0, int GB = 0, int EW = 4>
+__global__ void __launch_bounds__(tc_threads(CG, EW), 1)
     cell_tc_kernel(const __grid_constant__ CUtensorMap mapA0, const __grid_constant__ CUtensorMap mapA1,
                    const __grid_constant__ CUtensorMap mapW, const CellArgs a, int P) {
-  using C = TcCfg<MT, BN, STAGES, ACC, CG>;
+  using C = TcCfg<MT, BN, STAGES, ACC, CG, EW>;
+  static_assert(EW == 4 || (EW == 8 && CG == 1 && MODE != 1), "eight epilogue warps: cell tiles");
   constexpr bool PAIR = CG == 2;
-  constexpr int kGenWarps = gen_warps(CG);
+  constexpr int kGenWarps = gen_warps(CG, EW);
   constexpr int kGenThreads = kGenWarps * 32;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -450,7 +457,7 @@ __global__ void __launch_bounds__(tc_threads(CG), 1)
     }
     for (int b = 0; b < ACC; ++b) {
       mbar_init(accf_bar(b), 1);
-      mbar_init(acce_bar(b), 4 * CG);
+      mbar_init(acce_bar(b), EW * CG);
     }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -781,10 +788,14 @@ __global__ void __launch_bounds__(tc_threads(CG), 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int quad = warp & 3;
+    const int quad = warp & 3;                      // TMEM lane quadrant
+    const int ew = warp - 2 - kGenWarps;               // epilogue warp 0 .. EW-1
+    // units of the tile this warp finishes: all of them, or (EW = 8) one half
+    constexpr int UW = C::U * 4 / EW;
+    const int ubeg = (ew >> 2) * UW, uend = ubeg + UW;
     const int rloc = quad * 32 + lane;
     // this warp's copy of the tile's bias slice [4 gates][U units]
-    float* bias_s = reinterpret_cast<float*>(smem + STAGES * C::STAGE + 256) + quad * 4 * C::U;
+    float* bias_s = reinterpret_cast<float*>(smem + STAGES * C::STAGE + 256) + ew * 4 * C::U;
     uint32_t tcount = 0;
     bool ok = true;
     for (int64_t tile = walker; tile < a.tiles && ok; tile += walkers, ++tcount) {
@@ -809,14 +820,15 @@ __global__ void __launch_bounds__(tc_threads(CG), 1)
         for (int mt = 0; mt < MT; ++mt) {
           const int b = brow0 + mt * 128 + rloc;
           if (b < a.B) {
-            prefetch_l2(a.cst + ((int64_t)tc.ps * a.Bmax + b) * a.H + tc.n * C::U,
-                        C::U * (int)sizeof(float));
+            prefetch_l2(a.cst + ((int64_t)tc.ps * a.Bmax + b) * a.H + tc.n * C::U + ubeg,
+                        UW * (int)sizeof(float));
             if constexpr (MODE == 2) {
               const int tok = a.tokens[(int64_t)b * a.T + a.t];
               if (tok >= 0 && tok < a.V) {
-                const float* tr = a.vt + ((int64_t)tc.ps * a.vtrows + tok) * 4 * a.H + tc.n * C::U;
+                const float* tr =
+                    a.vt + ((int64_t)tc.ps * a.vtrows + tok) * 4 * a.H + tc.n * C::U + ubeg;
 #pragma unroll
-                for (int g = 0; g < 4; ++g) prefetch_l2(tr + g * a.H, C::U * (int)sizeof(float));
+                for (int g = 0; g < 4; ++g) prefetch_l2(tr + g * a.H, UW * (int)sizeof(float));
               }
             }
           }
@@ -889,15 +901,15 @@ __global__ void __launch_bounds__(tc_threads(CG), 1)
         constexpr bool kTwoAhead = MODE != 2;
         float4 cn0 = make_float4(0.f, 0.f, 0.f, 0.f), cn1 = cn0, cm0 = cn0, cm1 = cn0;
         if (need_c) {
-          cn0 = crow[0];
-          cn1 = crow[1];
-          if (kTwoAhead && 8 < C::U) {
-            cm0 = crow[2];
-            cm1 = crow[3];
+          cn0 = crow[(ubeg >> 2)];
+          cn1 = crow[(ubeg >> 2) + 1];
+          if (kTwoAhead && ubeg + 8 < uend) {
+            cm0 = crow[(ubeg >> 2) + 2];
+            cm1 = crow[(ubeg >> 2) + 3];
           }
         }
 #pragma unroll 1
-        for (int u0 = 0; u0 < C::U; u0 += 8) {
+        for (int u0 = ubeg; u0 < uend; u0 += 8) {
           // table loads issued before the TMEM loads: their latency overlaps the wait
           float4 tv[4][2];
           if constexpr (MODE == 2) {
@@ -919,11 +931,11 @@ __global__ void __launch_bounds__(tc_threads(CG), 1)
           if constexpr (kTwoAhead) {
             cn0 = cm0;
             cn1 = cm1;
-            if (need_c && u0 + 16 < C::U) {
+            if (need_c && u0 + 16 < uend) {
               cm0 = crow[(u0 >> 2) + 4];
               cm1 = crow[(u0 >> 2) + 5];
             }
-          } else if (need_c && u0 + 8 < C::U) {
+          } else if (need_c && u0 + 8 < uend) {
             cn0 = crow[(u0 >> 2) + 2];
             cn1 = crow[(u0 >> 2) + 3];
           }
@@ -1073,11 +1085,12 @@ bool make_cell_maps(zo_ctx* c) {
   return ok;
 }
 
-template <int MT, int BN, int STAGES, int ACC, int MODE, int CG, int XP = 0, int GB = 0>
+template <int MT, int BN, int STAGES, int ACC, int MODE, int CG, int XP = 0, int GB = 0,
+          int EW = 4>
 static cudaError_t launch_cfg(const CUtensorMap& A0, const CUtensorMap& A1, const CUtensorMap& Wm,
                               CellArgs a, int P, int sms, cudaStream_t st) {
-  using C = TcCfg<MT, BN, STAGES, ACC, CG>;
-  auto kern = cell_tc_kernel<MT, BN, STAGES, ACC, MODE, CG, XP, GB>;
+  using C = TcCfg<MT, BN, STAGES, ACC, CG, EW>;
+  auto kern = cell_tc_kernel<MT, BN, STAGES, ACC, MODE, CG, XP, GB, EW>;
   a.m_tiles = (a.B + C::ROWS - 1) / C::ROWS;
   a.n_tiles = MODE != 1 ? a.H / C::U : 1;
   a.tiles = (int64_t)P * a.m_tiles * a.n_tiles;
@@ -1085,7 +1098,7 @@ static cudaError_t launch_cfg(const CUtensorMap& A0, const CUtensorMap& A1, cons
   if (e != cudaSuccess) return e;
   if constexpr (CG == 1) {
     const int64_t grid = a.tiles < sms ? a.tiles : sms;
-    kern<<<(int)grid, tc_threads(CG), C::SMEM, st>>>(A0, A1, Wm, a, P);
+    kern<<<(int)grid, tc_threads(CG, EW), C::SMEM, st>>>(A0, A1, Wm, a, P);
     count_launch();
     return cudaGetLastError();
   } else {
@@ -1097,7 +1110,7 @@ static cudaError_t launch_cfg(const CUtensorMap& A0, const CUtensorMap& A1, cons
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
-    cfg.blockDim = dim3(tc_threads(CG), 1, 1);
+    cfg.blockDim = dim3(tc_threads(CG, EW), 1, 1);
     cfg.dynamicSmemBytes = C::SMEM;
     cfg.stream = st;
     cfg.attrs = attr;
@@ -1185,6 +1198,9 @@ cudaError_t launch_cell_tc(const zo_ctx* ctx, int layer, int t, int B, int nprob
     case ZO_CELL_PAIR_DIRECT_W:
       if (tab) return launch_cfg<1, 256, 6, 2, 2, 2, 0, 1>(A0, A1, Wm, a, P, sms, st);
       return launch_cfg<1, 256, 6, 2, 0, 2, 0, 1>(A0, A1, Wm, a, P, sms, st);
+    case ZO_CELL_SINGLE_EPI8:
+      if (tab) return launch_cfg<2, 256, 3, 1, 2, 1, 0, 0, 8>(A0, A1, Wm, a, P, sms, st);
+      return launch_cfg<2, 256, 3, 1, 0, 1, 0, 0, 8>(A0, A1, Wm, a, P, sms, st);
     default:
       // one CTA per 256 x 256 tile: two M = 128 MMAs per K slice on one B,
       // one accumulator, three 64 KB stages
@@ -1295,6 +1311,8 @@ cudaError_t launch_vocab_table(const zo_ctx* ctx, int nprobe, int probe0, uint64
       return launch_cfg<1, 256, 6, 2, 3, 2, 1>(m.x, m.x, m.w[0], a, P, sms, st);
     case ZO_CELL_PAIR_DIRECT_W:
       return launch_cfg<1, 256, 6, 2, 3, 2, 0, 1>(m.x, m.x, m.w[0], a, P, sms, st);
+    case ZO_CELL_SINGLE_EPI8:
+      return launch_cfg<2, 256, 3, 1, 3, 1, 0, 0, 8>(m.x, m.x, m.w[0], a, P, sms, st);
     default:
       return launch_cfg<2, 256, 3, 1, 3, 1>(m.x, m.x, m.w[0], a, P, sms, st);
   }

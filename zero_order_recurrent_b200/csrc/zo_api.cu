@@ -552,7 +552,7 @@ int zo_profile_read(zo_ctx* ctx, int32_t kind, int64_t* launches, double* total_
 }
 
 int zo_debug_cell_variant(zo_ctx* ctx, int32_t variant) {
-  if (!ctx || variant < ZO_CELL_SINGLE || variant > ZO_CELL_PAIR_DIRECT_W)
+  if (!ctx || variant < ZO_CELL_SINGLE || variant > ZO_CELL_SINGLE_EPI8)
     return ZO_ERR_INVALID_ARG;
   if (ctx->spec.dtype != ZO_DTYPE_BF16) return ZO_ERR_UNSUPPORTED;
   ctx->cell_variant = variant;
