@@ -41,12 +41,12 @@
 
 namespace zo {
 
-// generator warps: eight on single-CTA tiles (256 W rows per stage, one row a
-// thread), four on pair tiles (128 rows, still one row a thread)
+// generator warps: eight (one W row a thread on single-CTA tiles, half a row
+// on pair tiles)
 // (ew = 8 on single-CTA tiles: four generator warps, two rows a thread, and
 // eight epilogue warps, two per TMEM lane quadrant, each taking half the units)
 __host__ __device__ constexpr int gen_warps(int cg, int ew = 4) {
-  return cg == 2 ? 4 : (ew == 8 ? 4 : 8);
+  return ew == 8 ? 4 : 8;
 }
 __host__ __device__ constexpr int tc_threads(int cg, int ew = 4) {
   return (2 + gen_warps(cg, ew) + ew) * 32;
@@ -243,6 +243,18 @@ __device__ __forceinline__ void umma_commit(uint32_t bar) {
 }
 
 // ---- CTA-pair (cluster of two) forms -------------------------------------
+// cp.async.bulk of `bytes` (a multiple of 16, 16-byte aligned) from this CTA's
+// shared memory to `dst` in another CTA of the cluster, completing `bytes`
+// transactions on the barrier `bar` of that CTA (dst and bar: shared::cluster)
+__device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst, uint32_t src, uint32_t bytes,
+                                                  uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, "
+      "[%3];" ::"r"(dst),
+      "r"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
 __device__ __forceinline__ uint32_t cluster_rank() {
   uint32_t r;
   asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
@@ -383,7 +395,7 @@ struct TcCfg {
   static constexpr int COLS = MT * BN;              // TMEM columns per accumulator
   static constexpr int TMEM_COLS = COLS * ACC;
   static constexpr int EPI = EW * 4 * U * 4;         // per epilogue warp: bias slice [4][U]
-  static constexpr int SMEM = STAGES * STAGE + 1024 + 256 + EPI;
+  static constexpr int SMEM = STAGES * STAGE + 1024 + 512 + EPI;
   static_assert(BN % 64 == 0 && BN <= 256, "BN");
   static_assert(CG == 1 || (CG == 2 && MT == 1 && BN == 256), "pair tiles are 256 x 256");
   static_assert(TMEM_COLS == 128 || TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM columns");
@@ -429,6 +441,10 @@ __global__ void __launch_bounds__(tc_threads(CG, EW), 1)
   const uint32_t drain_bar = bar0 + 8u * (3 * STAGES + 2 * ACC);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * STAGES + 2 * ACC + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  // 16-byte handshake words, one per stage, at [bar0 + 256, bar0 + 256 + 16 STAGES)
+  auto hs_word = [&](int s) { return bar0 + 256u + 16u * s; };
+  static_assert(8 * (3 * STAGES + 2 * ACC + 1) + 8 <= 256 && 256 + 16 * STAGES <= 512,
+                "barrier area");
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -450,8 +466,9 @@ __global__ void __launch_bounds__(tc_threads(CG, EW), 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(full_bar(s), 1);
-      // CTA 1's generator warps arrive on their own barrier; one thread of
-      // CTA 1 forwards a single arrival per stage to CTA 0's
+      // CTA 1's generator warps arrive on their own barrier; CTA 0's counts
+      // its own generator warps and its producer, which also expects the 16
+      // bytes that CTA 1 copies in once its half of the stage is ready
       mbar_init(ready_bar(s), kGenWarps + (PAIR && rank == 0 ? 1 : 0));
       mbar_init(empty_bar(s), 1);
     }
@@ -527,6 +544,8 @@ __global__ void __launch_bounds__(tc_threads(CG, EW), 1)
                           g * a.gstride + tc.n * C::U);
             }
           }
+          // CTA 0: one arrival and the 16 bytes CTA 1's handshake copy brings
+          if (PAIR && rank == 0) mbar_expect_tx(ready_bar(s), 16);
         }
       }
       if (!ok) {
@@ -543,9 +562,12 @@ __global__ void __launch_bounds__(tc_threads(CG, EW), 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (PAIR && lane == 0 && rank == 1) {
-      // forwarder: once this CTA's generator warps have released a stage
-      // (CTA-scope arrivals on its own barrier), pass one cluster-scope
-      // arrival to CTA 0, whose MMA thread reads this CTA's half of the stage
+      // handshake: once this CTA's generator warps have perturbed their half
+      // of a stage (each fenced its writes for the async proxy and arrived on
+      // this CTA's barrier), copy 16 bytes into CTA 0 with cp.async.bulk; the
+      // copy's completion on CTA 0's barrier is what CTA 0's MMA thread waits
+      // for, the same async-proxy completion that a TMA load into one CTA
+      // signalling the other CTA's barrier uses - no cluster-wide fence
       uint32_t it = 0;
       bool ok = true;
       for (int64_t tile = walker; tile < a.tiles && ok; tile += walkers) {
@@ -555,7 +577,14 @@ __global__ void __launch_bounds__(tc_threads(CG, EW), 1)
             ok = false;
             break;
           }
-          mbar_arrive_cluster(peer_addr(ready_bar(s), 0));
+          bulk_copy_to_peer(peer_addr(hs_word(s), 0), hs_word(s), 16, peer_addr(ready_bar(s), 0));
+        }
+      }
+      // after an abort a copy may still be on its way into CTA 0: give it
+      // time to land before the cluster can exit
+      if (!ok) {
+        const uint64_t t0 = globaltimer();
+        while (globaltimer() - t0 < 50000ull) {
         }
       }
     }
@@ -792,10 +821,11 @@ __global__ void __launch_bounds__(tc_threads(CG, EW), 1)
     const int ew = warp - 2 - kGenWarps;               // epilogue warp 0 .. EW-1
     // units of the tile this warp finishes: all of them, or (EW = 8) one half
     constexpr int UW = C::U * 4 / EW;
-    const int ubeg = (ew >> 2) * UW, uend = ubeg + UW;
+    const int ubeg = EW == 8 ? (ew >> 2) * UW : 0;
+    const int uend = ubeg + UW;
     const int rloc = quad * 32 + lane;
     // this warp's copy of the tile's bias slice [4 gates][U units]
-    float* bias_s = reinterpret_cast<float*>(smem + STAGES * C::STAGE + 256) + ew * 4 * C::U;
+    float* bias_s = reinterpret_cast<float*>(smem + STAGES * C::STAGE + 512) + ew * 4 * C::U;
     uint32_t tcount = 0;
     bool ok = true;
     for (int64_t tile = walker; tile < a.tiles && ok; tile += walkers, ++tcount) {
@@ -1004,9 +1034,18 @@ __global__ void __launch_bounds__(tc_threads(CG, EW), 1)
 
   tc_fence_before();
   __syncthreads();
+  // after an abort, CTA 1's handshake copies may still be landing in CTA 0
+  if (PAIR && rank == 0 && threadIdx.x == 0 && *abort_flag) {
+    const uint64_t t0 = globaltimer();
+    while (globaltimer() - t0 < 50000ull) {
+    }
+  }
   // neither CTA of a pair leaves while the other may still read its shared
   // memory (MMA operands) or arrive on its barriers
-  if constexpr (PAIR) cluster_sync_all();
+  if constexpr (PAIR) {
+    __syncthreads();
+    cluster_sync_all();
+  }
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
