@@ -175,8 +175,9 @@ ZO_API int zo_coeffs_forward(zo_ctx* ctx, const float* loss_plus_dev, const floa
  * theta_dev is updated in place; padding stays zero.  For ZO_DTYPE_BF16 the
  * bf16 shadow is rewritten in the same pass.  If any coefficient is non-finite
  * theta is left unchanged and ZO_ERR_NONFINITE is latched.  n_pert is at
- * most ZO_MAX_UPDATE_PROBES (the kernel keeps 16 fp32 subset sums per four
- * probes in shared memory); larger counts return ZO_ERR_INVALID_ARG.  Async. */
+ * most ZO_MAX_UPDATE_PROBES (above 64 probes the kernel keeps 16 fp32 subset
+ * sums per four probes in shared memory); larger counts return
+ * ZO_ERR_INVALID_ARG.  Async. */
 #define ZO_MAX_UPDATE_PROBES 8192
 ZO_API int zo_update(zo_ctx* ctx, float* theta_dev, uint64_t step_seed, int32_t n_pert,
               const float* coeffs_dev, void* stream);

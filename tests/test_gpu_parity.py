@@ -101,12 +101,17 @@ def _check_update(cfg, n, theta, seed, coeffs, ctx, idx=None):
     return th
 
 
-# every probe-group count the update kernel compiles (1, 2, 4, 8, 16 groups of
-# four probes), counts that leave a group partly empty, and several passes
+# every probe-group count the update kernels compile (1 and 2 groups of four
+# probes up to 8 probes, 16 groups per pass above 64; 2, 4 and 8 groups of
+# eight for 9..64 probes), counts that leave a group partly empty, and
+# several passes
 @pytest.mark.parametrize("name,n", [("tiny", 8), ("tiny", 1), ("tiny", 3), ("overfit", 512),
-                                    ("overfit", 37), ("overfit", 5), ("overfit", 13),
-                                    ("overfit", 16), ("overfit", 29), ("overfit", 32),
-                                    ("overfit", 64), ("overfit", 65), ("overfit", 100)])
+                                    ("overfit", 37), ("overfit", 5), ("overfit", 9),
+                                    ("overfit", 13),
+                                    ("overfit", 16), ("overfit", 17), ("overfit", 29),
+                                    ("overfit", 32), ("overfit", 33), ("overfit", 48),
+                                    ("overfit", 64), ("overfit", 65), ("overfit", 100),
+                                    ("tiny", 24), ("tiny", 57)])
 def test_update_matches_oracle(name, n):
     cfg = W.CONFIGS[name]
     theta = W.init_theta(cfg)
@@ -167,13 +172,14 @@ def test_update_rejects_too_many_probes():
         assert torch.equal(th, dev(W.init_theta(cfg)))
 
 
-def test_update_bf16_context_sampled_and_shadow():
-    """charlm-size theta: sampled indices against the oracle; the bf16 shadow
-    the update writes equals a fresh cast of theta' (losses bit-identical)."""
+@pytest.mark.parametrize("n", [64, 32, 21, 12])
+def test_update_bf16_context_sampled_and_shadow(n):
+    """charlm-size theta (many spans per warp): sampled indices against the
+    oracle; the bf16 shadow the update writes equals a fresh cast of theta'
+    (losses bit-identical)."""
     cfg = W.CONFIGS["charlm"]
     theta = W.init_theta(cfg)
     seed = W.step_seed(1)
-    n = cfg.n_pert
     coeffs = np.random.default_rng(0).standard_normal(n) * 1e-4
     rng = np.random.default_rng(1)
     mask = O.real_mask(*spec_of(cfg))

@@ -110,8 +110,10 @@ cudaError_t launch_coeffs_forward(const float* lp, const float* l0, int n, float
 }
 
 // ---------------------------------------------------------------------------
-// Update.  theta'_j = theta_j + sum_i (-c_i) p_ij is evaluated four probes at
-// a time through subset-sum tables: for the probes 4g..4g+3 of group g,
+// Update with four-probe tables (up to 8 probes, and above 64 in passes of
+// 16 groups; 9..64 probes take the eight-probe tables below).
+// theta'_j = theta_j + sum_i (-c_i) p_ij is evaluated four probes at a time
+// through subset-sum tables: for the probes 4g..4g+3 of group g,
 //   T_g[s] = sum_{r<4} (-c_{4g+r}) (1 - 2 s_r),   s = 4-bit sign pattern,
 // (16 entries, computed in fp64 and rounded once) so one shared-memory lookup
 // replaces four sign applications.  The tables hold 16 consecutive words, one
@@ -185,6 +187,34 @@ __device__ __forceinline__ float table_at(const float* t, uint32_t byte_off) {
   return *reinterpret_cast<const float*>(reinterpret_cast<const char*>(t) + byte_off);
 }
 
+// theta' of block q (lane: its float4): pads past the block's segment end
+// keep theta, and the bf16 shadow gets the same values.  clean: the whole
+// span lies inside one segment's real entries, so no block needs the segment
+// search or the mask.
+__device__ __forceinline__ void store_block(const UpdateArgs& a, int64_t q, int lane, int& sg,
+                                            bool clean, float4 th, float4 o) {
+  if (!clean) {
+    while (sg + 1 < a.nseg && q * 128 >= a.seg_off[sg + 1]) ++sg;
+    const int64_t lim = a.seg_end[sg];
+    if (q * 128 + 128 > lim) {
+      const int64_t j = q * 128 + 4 * lane;
+      o.x = j + 0 < lim ? o.x : th.x;
+      o.y = j + 1 < lim ? o.y : th.y;
+      o.z = j + 2 < lim ? o.z : th.z;
+      o.w = j + 3 < lim ? o.w : th.w;
+    }
+  }
+  reinterpret_cast<float4*>(a.theta)[q * 32 + lane] = o;
+  if (a.shadow) {
+    __nv_bfloat162 lo = __floats2bfloat162_rn(o.x, o.y);
+    __nv_bfloat162 hi = __floats2bfloat162_rn(o.z, o.w);
+    uint2 pk;
+    pk.x = *reinterpret_cast<uint32_t*>(&lo);
+    pk.y = *reinterpret_cast<uint32_t*>(&hi);
+    reinterpret_cast<uint2*>(a.shadow)[q * 32 + lane] = pk;
+  }
+}
+
 // NG groups (4 NG probes) per pass.  MULTI: runtime number of passes, each
 // pass's fp32 tree sum added into an fp64 accumulator (n_pert > 64).
 template <int NG, bool MULTI>
@@ -242,31 +272,8 @@ __global__ void __launch_bounds__(kUpdWarps * 32, 4) update_kernel(const UpdateA
     }
     asm volatile("cp.async.commit_group;" ::: "memory");
   };
-  // theta' of block q: pads past the block's segment end keep theta, and the
-  // bf16 shadow gets the same values
-  // (clean: the whole span lies inside one segment's real entries, so no
-  // block needs the search or the mask)
   auto write_out = [&](int64_t q, int& sg, bool clean, float4 th, float4 o) {
-    if (!clean) {
-      while (sg + 1 < a.nseg && q * 128 >= a.seg_off[sg + 1]) ++sg;
-      const int64_t lim = a.seg_end[sg];
-      if (q * 128 + 128 > lim) {
-        const int64_t j = q * 128 + 4 * lane;
-        o.x = j + 0 < lim ? o.x : th.x;
-        o.y = j + 1 < lim ? o.y : th.y;
-        o.z = j + 2 < lim ? o.z : th.z;
-        o.w = j + 3 < lim ? o.w : th.w;
-      }
-    }
-    reinterpret_cast<float4*>(a.theta)[q * 32 + lane] = o;
-    if (a.shadow) {
-      __nv_bfloat162 lo = __floats2bfloat162_rn(o.x, o.y);
-      __nv_bfloat162 hi = __floats2bfloat162_rn(o.z, o.w);
-      uint2 pk;
-      pk.x = *reinterpret_cast<uint32_t*>(&lo);
-      pk.y = *reinterpret_cast<uint32_t*>(&hi);
-      reinterpret_cast<uint2*>(a.shadow)[q * 32 + lane] = pk;
-    }
+    store_block(a, q, lane, sg, clean, th, o);
   };
   int buf = 0;
   if (gw < nspan) issue(gw, stage);
@@ -386,6 +393,240 @@ static cudaError_t launch_update_ng(const UpdateArgs& a, int sm_count, cudaStrea
   return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------------------
+// Update with eight-probe tables (9..64 probes).  For the probes 8g..8g+7,
+//   T_g[s] = sum_{r<8} (-c_{8g+r}) (1 - 2 s_r),   s = 8-bit sign pattern,
+// so one lookup stands for eight sign applications, half the lookups and
+// tree adds of the four-probe tables.  256 entries read at random would
+// collide in the 32 banks, so every entry is stored 16 times: a 64 KB table
+// block B holds rows of 256 bytes (row e: entry e), and in each row the
+// groups 4B + t (t = 0..3) take bytes 64t..64t+63, one copy per 4 bytes.  In
+// one lookup, lanes 0..15 read group 4B + t from copy (lane & 15) and lanes
+// 16..31 read group 4B + ((t + 1) & 3), which sits in the other half of the
+// banks, so every lane hits its own bank.  The byte offset e * 256 is the
+// pattern byte itself moved to byte 1 of the address by one byte permute that
+// takes bytes 0, 2 and 3 from the lane's column word (the block base is 64 KB
+// aligned), so each lookup is one PRMT and one LDS.
+//
+// Sign phase: lane t owns one (group, block) pair, computes its eight probes'
+// Philox blocks, and per word position transposes the 8 x 32 bit matrix with
+// three rounds of delta swaps: byte q of word m then holds the eight probes'
+// bits at bit position 8q + m, the byte placement of the four-probe kernel,
+// so the apply phase picks a lane's bytes the same way.  Each warp owns a
+// slot (index rows and a theta staging buffer) in the shared memory
+// around the table blocks.
+// ---------------------------------------------------------------------------
+constexpr int kIdx8Row = 36;        // 32-bit words per (group, block) row: 32 + 4 pad
+constexpr int kUpd8MaxWarps = 16;   // 128 registers a thread
+
+// After the three rounds, bit r of byte q of x[m] is bit 8q + m of the input
+// x[r].  Round d exchanges, between x[i] and x[i + d] (i & d == 0), the bits
+// of x[i] at positions p with p & d set and those of x[i + d] at p - d: each
+// new word is one shift and one three-input select.
+__device__ __forceinline__ void transpose8x32(uint32_t (&x)[8]) {
+#pragma unroll
+  for (int d = 1; d < 8; d <<= 1) {
+    const uint32_t m = d == 1 ? 0x55555555u : d == 2 ? 0x33333333u : 0x0F0F0F0Fu;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (i & d) continue;
+      const uint32_t lo = bit_select(m, x[i], x[i + d] << d);
+      const uint32_t hi = bit_select(m, x[i] >> d, x[i + d]);
+      x[i] = lo;
+      x[i + d] = hi;
+    }
+  }
+}
+
+// Shared-memory load at addr + OFF (OFF: the table block's offset).
+template <int OFF>
+__device__ __forceinline__ float lds_table(uint32_t addr) {
+  float v;
+  asm("ld.shared.f32 %0, [%1+%2];" : "=f"(v) : "r"(addr), "n"(OFF));
+  return v;
+}
+
+// The four table values of a lane's four elements for one eight-probe group:
+// idx points at the lane's two index words in the group's row for the block.
+template <int OFF>
+__device__ __forceinline__ void lookup8(const uint32_t* idx, uint32_t col, uint32_t sel_lo,
+                                        uint32_t sel_hi, float2& v01, float2& v23) {
+  const uint2 wv = *reinterpret_cast<const uint2*>(idx);
+  v01.x = lds_table<OFF>(__byte_perm(wv.x, col, sel_lo));
+  v01.y = lds_table<OFF>(__byte_perm(wv.x, col, sel_hi));
+  v23.x = lds_table<OFF>(__byte_perm(wv.y, col, sel_lo));
+  v23.y = lds_table<OFF>(__byte_perm(wv.y, col, sel_hi));
+}
+
+// A span's theta copies are issued when the span starts and fly during its
+// sign phase; one staging buffer keeps the slot small, so 16 warps fit (with
+// two buffers, the next span's copies in flight during this span, only 12 fit
+// at 32 probes and 6 at 16, and the kernel ran 8-24% slower).
+template <int G8>
+__global__ void __launch_bounds__(kUpd8MaxWarps * 32, 1)
+    update8_kernel(const UpdateArgs a, uint32_t dyn_bytes) {
+  constexpr int S = 32 / G8;            // blocks per span: G8 x S (group, block) pairs = 32 lanes
+  constexpr int NB = (G8 + 3) / 4;      // 64 KB table blocks
+  constexpr int KG = G8 < 4 ? G8 : 4;   // groups per table block
+  constexpr uint32_t kIdxBytes = 32 * kIdx8Row * 4;
+  constexpr uint32_t kSlot = kIdxBytes + S * 512;
+  static_assert(G8 == 2 || G8 == 4 || G8 == 8, "eight-probe tables: 2, 4 or 8 groups");
+  extern __shared__ __align__(16) unsigned char dyn[];
+  const uint32_t base = (uint32_t)__cvta_generic_to_shared(dyn);
+  const uint32_t t0 = (base + 0xFFFFu) & ~0xFFFFu;
+  const uint32_t tend = t0 + NB * 65536u;
+  if (tend > base + dyn_bytes) {   // the launcher sizes the allocation so this cannot happen
+    if (threadIdx.x == 0) latch(a.err, kErrBounds);
+    return;
+  }
+  bool badc = false;
+  for (int e = threadIdx.x; e < G8 * 256; e += blockDim.x) {
+    const int g = e >> 8, s = e & 255;
+    double t = 0.0;
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const int i = 8 * g + r;
+      const float c = i < a.n ? a.coeffs[i] : 0.f;
+      badc |= !isfinite(c);
+      t += ((s >> r) & 1) ? (double)c : -(double)c;
+    }
+    const float v = (float)t;
+    float4* row = reinterpret_cast<float4*>(dyn + (t0 - base) + (g / KG) * 65536 + s * 256 +
+                                            (g % KG) * 64);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) row[k] = make_float4(v, v, v, v);
+  }
+  if (__syncthreads_or(badc)) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) latch(a.err, kErrNonfinite);
+    return;
+  }
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int nwarps = blockDim.x >> 5;
+  const uint32_t nfront = (t0 - base) / kSlot;
+  const uint32_t slot = (uint32_t)warp < nfront ? base + warp * kSlot
+                                                : tend + ((uint32_t)warp - nfront) * kSlot;
+  if (slot + kSlot > base + dyn_bytes) {   // likewise excluded by the launcher
+    if (lane == 0) latch(a.err, kErrBounds);
+    return;
+  }
+  uint32_t* idxw = reinterpret_cast<uint32_t*>(dyn + (slot - base));
+  const float4* stage = reinterpret_cast<const float4*>(dyn + (slot - base) + kIdxBytes);
+  const uint32_t stage_s = slot + kIdxBytes;
+  const int64_t nspan = (a.nblk + S - 1) / S;
+  const int64_t gw = blockIdx.x * (int64_t)nwarps + warp;
+  const int64_t nw = (int64_t)gridDim.x * nwarps;
+  const float4* th4 = reinterpret_cast<const float4*>(a.theta);
+  // apply role: as in the four-probe kernel, elements 4m..4m+3 of word
+  // lane>>3 (m = lane & 7) take bytes (m>>2, m>>2 + 2) of words 2(m&3), +1;
+  // the permute puts the byte at bits 8..15 over the column word
+  const int unit = (lane >> 3) * 4 + (lane & 3);
+  const uint32_t sel_lo = 0x7604u | ((uint32_t)((lane & 7) >> 2) << 4);
+  const uint32_t sel_hi = sel_lo + 0x20u;
+  uint32_t col[KG];
+  int rowoff[KG];
+#pragma unroll
+  for (int k = 0; k < KG; ++k) {
+    const int t = (k + (lane >> 4)) & (KG - 1);
+    col[k] = t0 + 4u * (uint32_t)((lane & 15) + 16 * t);
+    rowoff[k] = t * S * kIdx8Row + 2 * unit;
+  }
+  const int pg = lane / S, pb = lane % S;   // sign role: this lane's (group, block) pair
+
+  auto issue = [&](int64_t sp) {
+    const int64_t qq = sp * S;
+    const int nn = (int)min((int64_t)S, a.nblk - qq);
+    for (int it = 0; it < nn; ++it) {
+      const uint32_t dst = stage_s + (uint32_t)((it * 32 + lane) * 16);
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst),
+                   "l"(th4 + (qq + it) * 32 + lane)
+                   : "memory");
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+  for (int64_t span = gw; span < nspan; span += nw) {
+    const int64_t q0 = span * S;
+    const int nq = (int)min((int64_t)S, a.nblk - q0);
+    issue(span);
+    int sg = 0;
+    while (sg + 1 < a.nseg && q0 * 128 >= a.seg_off[sg + 1]) ++sg;
+    const bool clean = (q0 + nq) * 128 <= a.seg_end[sg];
+    // sign phase (probes past n_pert have zero coefficients, so their bits
+    // select equal table entries and need no masking)
+    if (pb < nq) {
+      uint4 w[8];
+#pragma unroll
+      for (int r = 0; r < 8; ++r)
+        w[r] = sign_block(a.seed, (uint32_t)(8 * pg + r), (uint64_t)(q0 + pb));
+      uint32_t* row = idxw + lane * kIdx8Row;
+#pragma unroll
+      for (int wi = 0; wi < 4; ++wi) {
+        uint32_t x[8];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) x[r] = word_of(w[r], wi);
+        transpose8x32(x);
+        reinterpret_cast<uint4*>(row + wi * 8)[0] = make_uint4(x[0], x[1], x[2], x[3]);
+        reinterpret_cast<uint4*>(row + wi * 8)[1] = make_uint4(x[4], x[5], x[6], x[7]);
+      }
+    }
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+    __syncwarp();
+    // apply phase
+#pragma unroll
+    for (int it = 0; it < S; ++it) {
+      if (it < nq) {
+        float2 v01[G8], v23[G8];
+#pragma unroll
+        for (int k = 0; k < KG; ++k) {
+          lookup8<0>(idxw + it * kIdx8Row + rowoff[k], col[k], sel_lo, sel_hi, v01[k], v23[k]);
+          if constexpr (NB == 2)
+            lookup8<65536>(idxw + (4 * S + it) * kIdx8Row + rowoff[k], col[k], sel_lo, sel_hi,
+                           v01[4 + k], v23[4 + k]);
+        }
+#pragma unroll
+        for (int w = 1; w < G8; w *= 2) {
+#pragma unroll
+          for (int g = 0; g + w < G8; g += 2 * w) {
+            v01[g] = add_f32x2(v01[g], v01[g + w]);
+            v23[g] = add_f32x2(v23[g], v23[g + w]);
+          }
+        }
+        const float4 th = stage[it * 32 + lane];
+        const float2 o01 = add_f32x2(make_float2(th.x, th.y), v01[0]);
+        const float2 o23 = add_f32x2(make_float2(th.z, th.w), v23[0]);
+        store_block(a, q0 + it, lane, sg, clean, th, make_float4(o01.x, o01.y, o23.x, o23.y));
+      }
+    }
+    __syncwarp();   // the next span's sign phase and copies reuse the slot
+  }
+}
+
+template <int G8>
+static cudaError_t launch_update8(const UpdateArgs& a, int sm_count, cudaStream_t st) {
+  constexpr int S = 32 / G8;
+  constexpr uint32_t kSlot = 32 * kIdx8Row * 4 + S * 512;
+  constexpr uint32_t kTables = ((G8 + 3) / 4) * 65536u;
+  int dev = 0, optin = 0;
+  cudaGetDevice(&dev);
+  if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+    return cudaErrorInvalidValue;
+  // the table blocks start at the first 64 KB boundary at or after the
+  // allocation's base: the slots fit in the two pieces around them, each
+  // piece losing less than one slot to the cut
+  const uint32_t dyn = (uint32_t)optin;
+  if (dyn < kTables + 65536u) return cudaErrorInvalidValue;
+  int warps = (int)((dyn - kTables) / kSlot) - 1;
+  if (warps > kUpd8MaxWarps) warps = kUpd8MaxWarps;
+  if (warps < 1) return cudaErrorInvalidValue;
+  cudaFuncSetAttribute(update8_kernel<G8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);
+  const int64_t nspan = (a.nblk + S - 1) / S;
+  int64_t grid = (nspan + warps - 1) / warps;
+  if (grid > sm_count) grid = sm_count;
+  update8_kernel<G8><<<(int)grid, warps * 32, dyn, st>>>(a, dyn);
+  count_launch();
+  return cudaGetLastError();
+}
+
 cudaError_t launch_update(const zo_ctx* ctx, float* theta, uint64_t seed, int n,
                           const float* coeffs, __nv_bfloat16* shadow, cudaStream_t st) {
   UpdateArgs a;
@@ -401,18 +642,21 @@ cudaError_t launch_update(const zo_ctx* ctx, float* theta, uint64_t seed, int n,
     a.seg_end[s] = ctx->seg.off[s] + ctx->seg.numel[s];
   }
   a.err = ctx->err;
-  const int ng = (n + 3) / 4;
-  if (ng <= 16) {
-    const int NG = ng <= 1 ? 1 : ng <= 2 ? 2 : ng <= 4 ? 4 : ng <= 8 ? 8 : 16;
-    a.ngroups = NG;
+  if (n > 8 && n <= 64) {
     a.chunks = 1;
-    switch (NG) {
-      case 1: return launch_update_ng<1, false>(a, ctx->sm_count, st);
-      case 2: return launch_update_ng<2, false>(a, ctx->sm_count, st);
-      case 4: return launch_update_ng<4, false>(a, ctx->sm_count, st);
-      case 8: return launch_update_ng<8, false>(a, ctx->sm_count, st);
-      default: return launch_update_ng<16, false>(a, ctx->sm_count, st);
-    }
+    a.ngroups = 0;
+    if (n <= 16) return launch_update8<2>(a, ctx->sm_count, st);
+    if (n <= 32) return launch_update8<4>(a, ctx->sm_count, st);
+    return launch_update8<8>(a, ctx->sm_count, st);
+  }
+  // up to 8 probes (one or two four-probe groups), and above 64 in passes
+  // of 16 four-probe groups
+  const int ng = (n + 3) / 4;
+  if (ng <= 2) {
+    a.ngroups = ng;
+    a.chunks = 1;
+    return ng == 1 ? launch_update_ng<1, false>(a, ctx->sm_count, st)
+                   : launch_update_ng<2, false>(a, ctx->sm_count, st);
   }
   a.chunks = (ng + 15) / 16;
   a.ngroups = a.chunks * 16;
