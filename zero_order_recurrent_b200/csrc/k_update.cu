@@ -533,21 +533,52 @@ __global__ void __launch_bounds__(kUpd8MaxWarps * 32, 1)
   }
   const int pg = lane / S, pb = lane % S;   // sign role: this lane's (group, block) pair
 
-  auto issue = [&](int64_t sp) {
-    const int64_t qq = sp * S;
-    const int nn = (int)min((int64_t)S, a.nblk - qq);
-    for (int it = 0; it < nn; ++it) {
-      const uint32_t dst = stage_s + (uint32_t)((it * 32 + lane) * 16);
-      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst),
-                   "l"(th4 + (qq + it) * 32 + lane)
-                   : "memory");
+  // theta copies of a span: lane's float4 of each block (full spans unrolled)
+  auto issue = [&](int64_t q0, int nq) {
+    const float4* src = th4 + q0 * 32 + lane;
+    const uint32_t dst = stage_s + (uint32_t)lane * 16u;
+    if (nq == S) {
+#pragma unroll
+      for (int it = 0; it < S; ++it)
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst + it * 512),
+                     "l"(src + it * 32)
+                     : "memory");
+    } else {
+      for (int it = 0; it < nq; ++it)
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst + it * 512),
+                     "l"(src + it * 32)
+                     : "memory");
     }
     asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+  // sum over the probes of block it's table values for this lane's four
+  // elements, plus theta
+  auto block_out = [&](int it, float4& th) -> float4 {
+    float2 v01[G8], v23[G8];
+#pragma unroll
+    for (int k = 0; k < KG; ++k) {
+      lookup8<0>(idxw + it * kIdx8Row + rowoff[k], col[k], sel_lo, sel_hi, v01[k], v23[k]);
+      if constexpr (NB == 2)
+        lookup8<65536>(idxw + (4 * S + it) * kIdx8Row + rowoff[k], col[k], sel_lo, sel_hi,
+                       v01[4 + k], v23[4 + k]);
+    }
+#pragma unroll
+    for (int w = 1; w < G8; w *= 2) {
+#pragma unroll
+      for (int g = 0; g + w < G8; g += 2 * w) {
+        v01[g] = add_f32x2(v01[g], v01[g + w]);
+        v23[g] = add_f32x2(v23[g], v23[g + w]);
+      }
+    }
+    th = stage[it * 32 + lane];
+    const float2 o01 = add_f32x2(make_float2(th.x, th.y), v01[0]);
+    const float2 o23 = add_f32x2(make_float2(th.z, th.w), v23[0]);
+    return make_float4(o01.x, o01.y, o23.x, o23.y);
   };
   for (int64_t span = gw; span < nspan; span += nw) {
     const int64_t q0 = span * S;
     const int nq = (int)min((int64_t)S, a.nblk - q0);
-    issue(span);
+    issue(q0, nq);
     int sg = 0;
     while (sg + 1 < a.nseg && q0 * 128 >= a.seg_off[sg + 1]) ++sg;
     const bool clean = (q0 + nq) * 128 <= a.seg_end[sg];
@@ -571,30 +602,28 @@ __global__ void __launch_bounds__(kUpd8MaxWarps * 32, 1)
     }
     asm volatile("cp.async.wait_group 0;" ::: "memory");
     __syncwarp();
-    // apply phase
+    // apply phase: a full span inside one segment's real entries with the
+    // shadow present (all but a few spans) stores without per-block checks
+    if (nq == S && clean && a.shadow) {
+      float4* tdst = reinterpret_cast<float4*>(a.theta) + q0 * 32 + lane;
+      uint2* sdst = reinterpret_cast<uint2*>(a.shadow) + q0 * 32 + lane;
 #pragma unroll
-    for (int it = 0; it < S; ++it) {
-      if (it < nq) {
-        float2 v01[G8], v23[G8];
+      for (int it = 0; it < S; ++it) {
+        float4 th;
+        const float4 o = block_out(it, th);
+        tdst[it * 32] = o;
+        __nv_bfloat162 lo = __floats2bfloat162_rn(o.x, o.y);
+        __nv_bfloat162 hi = __floats2bfloat162_rn(o.z, o.w);
+        sdst[it * 32] = make_uint2(*reinterpret_cast<uint32_t*>(&lo), *reinterpret_cast<uint32_t*>(&hi));
+      }
+    } else {
 #pragma unroll
-        for (int k = 0; k < KG; ++k) {
-          lookup8<0>(idxw + it * kIdx8Row + rowoff[k], col[k], sel_lo, sel_hi, v01[k], v23[k]);
-          if constexpr (NB == 2)
-            lookup8<65536>(idxw + (4 * S + it) * kIdx8Row + rowoff[k], col[k], sel_lo, sel_hi,
-                           v01[4 + k], v23[4 + k]);
+      for (int it = 0; it < S; ++it) {
+        if (it < nq) {
+          float4 th;
+          const float4 o = block_out(it, th);
+          store_block(a, q0 + it, lane, sg, clean, th, o);
         }
-#pragma unroll
-        for (int w = 1; w < G8; w *= 2) {
-#pragma unroll
-          for (int g = 0; g + w < G8; g += 2 * w) {
-            v01[g] = add_f32x2(v01[g], v01[g + w]);
-            v23[g] = add_f32x2(v23[g], v23[g + w]);
-          }
-        }
-        const float4 th = stage[it * 32 + lane];
-        const float2 o01 = add_f32x2(make_float2(th.x, th.y), v01[0]);
-        const float2 o23 = add_f32x2(make_float2(th.z, th.w), v23[0]);
-        store_block(a, q0 + it, lane, sg, clean, th, make_float4(o01.x, o01.y, o23.x, o23.y));
       }
     }
     __syncwarp();   // the next span's sign phase and copies reuse the slot
