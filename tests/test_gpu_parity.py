@@ -332,6 +332,33 @@ def test_nonfinite_loss_keeps_theta():
         assert np.array_equal(got[~np.isnan(theta)], theta[~np.isnan(theta)])
 
 
+@pytest.mark.parametrize("n,bad", [(3, float("nan")), (12, float("inf")), (24, float("nan")),
+                                   (64, float("-inf")), (100, float("nan"))])
+def test_update_nonfinite_coefficient_keeps_theta(n, bad):
+    """A non-finite coefficient leaves theta (and its bf16 shadow) unchanged and
+    latches ZO_ERR_NONFINITE, in each update kernel (four-probe tables, two,
+    four and eight eight-probe tables, four-probe passes)."""
+    cfg = W.CONFIGS["charlm"]
+    theta = W.init_theta(cfg)
+    coeffs = (np.random.default_rng(n).standard_normal(n) * 1e-3).astype(np.float32)
+    coeffs[n // 2] = bad
+    tok, tgt = W.markov_batch(128, 2, step=3)
+    with zo.Context.for_config(cfg, max_batch=128, max_seq=2, chunk=2) as ctx:
+        th = dev(theta)
+        lp0 = torch.empty(2, device="cuda")
+        lm0 = torch.empty(2, device="cuda")
+        zo.zo_probe_losses(ctx, th, 5, 2, cfg.eps, dev(tok), dev(tgt), lp0, lm0)
+        zo.zo_update(ctx, th, 5, n, dev(coeffs))
+        assert zo.zo_sync_status(ctx) == zo.ZO_ERR_NONFINITE
+        assert np.array_equal(th.cpu().numpy(), theta)
+        # the shadow still matches theta: the losses repeat bit for bit
+        lp1 = torch.empty(2, device="cuda")
+        lm1 = torch.empty(2, device="cuda")
+        zo.zo_probe_losses(ctx, th, 5, 2, cfg.eps, dev(tok), dev(tgt), lp1, lm1)
+        assert zo.zo_sync_status(ctx) == zo.ZO_OK
+        assert torch.equal(lp0, lp1) and torch.equal(lm0, lm1)
+
+
 def test_host_step_matches_device_step():
     cfg = W.CONFIGS["tiny"]
     theta = W.init_theta(cfg)
