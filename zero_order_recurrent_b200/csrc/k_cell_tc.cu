@@ -120,22 +120,13 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Memory scope of the pair's cross-CTA barrier traffic: 1 = release/acquire
-// at cluster scope; 0 = the default (CTA-scope) forms of arrive and wait on
-// the remote barrier.
-#ifndef ZO_PAIR_SYNC_CLUSTER
-#define ZO_PAIR_SYNC_CLUSTER 1
-#endif
-
+// Waits on a barrier that the other CTA of a pair arrives on: acquire at
+// cluster scope, pairing with the release of mbar_arrive_cluster.
 __device__ __forceinline__ bool mbar_try_cluster(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-#if ZO_PAIR_SYNC_CLUSTER
       "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-#else
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-#endif
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
       : "r"(bar), "r"(parity)
@@ -279,14 +270,10 @@ __device__ __forceinline__ uint32_t peer_addr(uint32_t addr, uint32_t rank) {
 }
 
 
-// arrive on a barrier of the cluster (here: CTA 0's)
+// arrive on a barrier of the cluster (here: CTA 0's), releasing at cluster scope
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-#if ZO_PAIR_SYNC_CLUSTER
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
                : "memory");
-#else
-  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
-#endif
 }
 
 __device__ __forceinline__ void cluster_sync_all() {
