@@ -68,7 +68,7 @@ struct CellArgs {
   int64_t offW;    // theta offset of W_l (Philox element index base)
   const float* small_p;   // perturbed small segments
   int64_t sstride, soffb; // per probe-sign stride, offset of b_l
-  float* cst;      // [P][Bmax][H] fp32
+  float* cst;      // fp32; [P][cst_rows(Bmax)/128][H/4][128][4], MODE 2: [P][Bmax][H]
   __nv_bfloat16* hout;    // [P][Bmax][H]
   int first;       // t == 0: c_{-1} = 0
   float* raw;      // optional [P][Bmax][4H] pre-activations (then c, h are not written)
@@ -87,6 +87,16 @@ struct CellArgs {
   uint64_t wait_ns;        // bound of every mbarrier wait
   int stall;               // test hook: the producer issues nothing (all waits run out)
 };
+
+// Cell state of units u.. (u a multiple of 4) in the 128-row block that starts
+// at batch row b0 of probe-sign ps: the state is stored
+// [ps][row/128][unit/4][row%128][4] floats, so a warp's 32 consecutive rows
+// of one four-unit group are 512 contiguous bytes.
+__device__ __forceinline__ float* cst_quad(const CellArgs& a, int ps, int b0, int u) {
+  const uint32_t nb = (uint32_t)(a.Bmax + 127) >> 7;
+  const uint32_t q = ((uint32_t)ps * nb + ((uint32_t)b0 >> 7)) * ((uint32_t)a.H >> 2) + ((uint32_t)u >> 2);
+  return a.cst + ((uint64_t)q << 9);
+}
 
 // ---------------------------------------------------------------------------
 // PTX wrappers
@@ -331,6 +341,15 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
 
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// After tmem_wait_ld: ties each register a tcgen05.ld wrote to a point after
+// the wait (the load defines them only asynchronously), so no read of them
+// can be scheduled before it.  Emits no instruction.
+template <int N>
+__device__ __forceinline__ void tmem_regs_ready(uint32_t* r) {
+#pragma unroll
+  for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i]));
 }
 
 __device__ __forceinline__ float tanh_fast(float x) {
@@ -837,8 +856,14 @@ __global__ void __launch_bounds__(tc_threads(CG, EW), 1)
         for (int mt = 0; mt < MT; ++mt) {
           const int b = brow0 + mt * 128 + rloc;
           if (b < a.B) {
-            prefetch_l2(a.cst + ((int64_t)tc.ps * a.Bmax + b) * a.H + tc.n * C::U + ubeg,
-                        UW * (int)sizeof(float));
+            // the block's units [ubeg, ubeg + UW) are one contiguous run of
+            // UW x 128 floats; each of the 128 rows' threads pulls 1/128 of it
+            if constexpr (MODE == 2)
+              prefetch_l2(a.cst + ((int64_t)tc.ps * a.Bmax + b) * a.H + tc.n * C::U + ubeg,
+                          UW * (int)sizeof(float));
+            else
+              prefetch_l2(cst_quad(a, tc.ps, b - rloc, tc.n * C::U + ubeg) + rloc * UW,
+                          UW * (int)sizeof(float));
             if constexpr (MODE == 2) {
               const int tok = a.tokens[(int64_t)b * a.T + a.t];
               if (tok >= 0 && tok < a.V) {
@@ -869,6 +894,7 @@ __global__ void __launch_bounds__(tc_threads(CG, EW), 1)
                       zq);
           }
           tmem_wait_ld();
+          tmem_regs_ready<BN>(z);
           if (b < a.B) {
             int tg = a.targets[(int64_t)b * a.T + a.t];
             if (tg >= a.V || tg < -1) {
@@ -899,7 +925,15 @@ __global__ void __launch_bounds__(tc_threads(CG, EW), 1)
         const int64_t rowoff = ((int64_t)tc.ps * a.Bmax + b) * a.H;
         const bool live = b < a.B;
         const bool need_c = live && !a.first && !a.raw;
-        float4* crow = reinterpret_cast<float4*>(a.cst + rowoff + tc.n * C::U);
+        // this row's c: units 4q..4q+3 of the tile at crow[q * QS].  Layer 0
+        // from the vocabulary table (MODE 2, whose table values fill the
+        // registers the four-unit layout's address arithmetic would need)
+        // keeps c row-major, [ps][row][unit]
+        constexpr int QS = MODE == 2 ? 1 : 128;
+        float4* crow =
+            MODE == 2
+                ? reinterpret_cast<float4*>(a.cst + rowoff + tc.n * C::U)
+                : reinterpret_cast<float4*>(cst_quad(a, tc.ps, b - rloc, tc.n * C::U)) + rloc;
         // input term from the vocabulary table: the row of this batch row's token
         const float* trow = nullptr;
         if constexpr (MODE == 2) {
@@ -918,11 +952,11 @@ __global__ void __launch_bounds__(tc_threads(CG, EW), 1)
         constexpr bool kTwoAhead = MODE != 2;
         float4 cn0 = make_float4(0.f, 0.f, 0.f, 0.f), cn1 = cn0, cm0 = cn0, cm1 = cn0;
         if (need_c) {
-          cn0 = crow[(ubeg >> 2)];
-          cn1 = crow[(ubeg >> 2) + 1];
+          cn0 = crow[(ubeg >> 2) * QS];
+          cn1 = crow[((ubeg >> 2) + 1) * QS];
           if (kTwoAhead && ubeg + 8 < uend) {
-            cm0 = crow[(ubeg >> 2) + 2];
-            cm1 = crow[(ubeg >> 2) + 3];
+            cm0 = crow[((ubeg >> 2) + 2) * QS];
+            cm1 = crow[((ubeg >> 2) + 3) * QS];
           }
         }
 #pragma unroll 1
@@ -949,14 +983,15 @@ __global__ void __launch_bounds__(tc_threads(CG, EW), 1)
             cn0 = cm0;
             cn1 = cm1;
             if (need_c && u0 + 16 < uend) {
-              cm0 = crow[(u0 >> 2) + 4];
-              cm1 = crow[(u0 >> 2) + 5];
+              cm0 = crow[((u0 >> 2) + 4) * QS];
+              cm1 = crow[((u0 >> 2) + 5) * QS];
             }
           } else if (need_c && u0 + 8 < uend) {
-            cn0 = crow[(u0 >> 2) + 2];
-            cn1 = crow[(u0 >> 2) + 3];
+            cn0 = crow[((u0 >> 2) + 2) * QS];
+            cn1 = crow[((u0 >> 2) + 3) * QS];
           }
           tmem_wait_ld();
+          tmem_regs_ready<32>(&acc[0][0]);
           if (live) {
             const int unit0 = tc.n * C::U + u0;
             float pre[4][8];
@@ -1006,8 +1041,8 @@ __global__ void __launch_bounds__(tc_threads(CG, EW), 1)
                 __nv_bfloat162 pr = __floats2bfloat162_rn(hv[0], hv[1]);
                 hp[i >> 1] = *reinterpret_cast<uint32_t*>(&pr);
               }
-              crow[(u0 >> 2)] = make_float4(cn[0], cn[1], cn[2], cn[3]);
-              crow[(u0 >> 2) + 1] = make_float4(cn[4], cn[5], cn[6], cn[7]);
+              crow[(u0 >> 2) * QS] = make_float4(cn[0], cn[1], cn[2], cn[3]);
+              crow[((u0 >> 2) + 1) * QS] = make_float4(cn[4], cn[5], cn[6], cn[7]);
               *reinterpret_cast<uint4*>(a.hout + rowoff + unit0) = make_uint4(hp[0], hp[1], hp[2], hp[3]);
             }
           }
@@ -1192,7 +1227,7 @@ cudaError_t launch_cell_tc(const zo_ctx* ctx, int layer, int t, int B, int nprob
   a.sstride = ctx->small.stride;
   a.soffb = ctx->small.b[layer];
   const int64_t PB = 2 * (int64_t)ctx->chunk * s.max_batch;
-  a.cst = ctx->cst + (int64_t)layer * PB * H;
+  a.cst = ctx->cst + (int64_t)layer * 2 * ctx->chunk * cst_rows(s.max_batch) * H;
   a.hout = ctx->h + ((int64_t)layer * 2 + (t & 1)) * PB * H;
   a.first = t == 0;
   a.raw = raw_out;

@@ -154,7 +154,7 @@ __global__ void vocab_first_kernel(const float* __restrict__ vt, int vtrows,
     const float og = sigmoid_ap(tr[3 * H + u] + bias[3 * H + u]);
     const float c = ig * gg;
     const int64_t o = ((int64_t)ps * Bmax + b) * H + u;
-    cst[o] = c;
+    cst[o] = c;   // row-major, as the table-fed layer's cell step reads it
     hout[o] = __float2bfloat16_rn(og * tanh_ap(c));
   }
 }

@@ -239,7 +239,7 @@ int zo_create(const zo_model_spec* spec, zo_ctx** out) {
     // batch row) costs less than the input K stages it replaces (2 E flops),
     // and the vocabulary rows fit one 256-row tile of the x buffer
     c->vocab = E >= 512 && B >= 256;
-    const int64_t per_ps = 2 * B * E + L * 2 * B * H * 2 + L * B * H * 4 + sl.stride * 4 + B * 4 +
+    const int64_t per_ps = 2 * B * E + L * 2 * B * H * 2 + L * cst_rows(B) * H * 4 + sl.stride * 4 + B * 4 +
                            (c->vocab ? (int64_t)kVocabRows * 4 * H * 4 : 0);
     int chunk = s.chunk;
     if (chunk == 0) {
@@ -255,7 +255,7 @@ int zo_create(const zo_model_spec* spec, zo_ctx** out) {
     alloc((void**)&c->small_p, sizeof(float) * P * sl.stride);
     alloc((void**)&c->x, sizeof(__nv_bfloat16) * P * B * E);
     alloc((void**)&c->h, sizeof(__nv_bfloat16) * L * 2 * P * B * H);
-    alloc((void**)&c->cst, sizeof(float) * L * P * B * H);
+    alloc((void**)&c->cst, sizeof(float) * L * P * cst_rows(B) * H);
     alloc((void**)&c->rowloss, sizeof(float) * P * B);
     if (c->vocab) alloc((void**)&c->vt, sizeof(float) * P * kVocabRows * 4 * H);
     if (rc == ZO_OK && !make_cell_maps(c)) rc = ZO_ERR_CUDA;

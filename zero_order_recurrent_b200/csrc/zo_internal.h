@@ -48,6 +48,14 @@ struct ZoProfRec {
   double flops = 0, bytes = 0;
 };
 
+// Rows of the fp32 cell-state buffer per probe-sign: the batch rounded up to
+// the 128-row blocks of its layout.  Within a block the state is stored four
+// units at a time, row-minor ([unit/4][row][4]), so the 32 lanes of a warp,
+// which hold 32 consecutive rows of one tensor-memory quadrant, read and write
+// 512 contiguous bytes.  A layer whose input term comes from the vocabulary
+// table keeps it row-major ([row][unit]).
+inline int64_t cst_rows(int64_t B) { return (B + 127) / 128 * 128; }
+
 struct zo_ctx {
   zo_model_spec spec;
   int device = 0;
@@ -64,7 +72,8 @@ struct zo_ctx {
   float* small_p = nullptr;      // [2*chunk][small.stride]
   __nv_bfloat16* x = nullptr;    // [2*chunk][B][E]
   __nv_bfloat16* h = nullptr;    // [L][2][2*chunk][B][H]
-  float* cst = nullptr;          // [L][2*chunk][B][H]
+  float* cst = nullptr;          // [L][2*chunk][cst_rows(B)*H]: [Bpad/128][H/4][128][4], or
+                                 // [B][H] for a layer fed by the vocabulary table
   zo::CellMaps* maps = nullptr;  // host copy of the tensor maps
   // vocabulary table of the first layer's input term (bf16 path, wide
   // embeddings): vt[ps][v][4H] = E'_ps[v] (W_0x +- eps P)^T, built once per chunk
