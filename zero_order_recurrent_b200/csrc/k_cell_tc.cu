@@ -1218,7 +1218,11 @@ cudaError_t launch_cell_tc(const zo_ctx* ctx, int layer, int t, int B, int nprob
   a.tokens = tokens;
   a.B = B;
   a.Bmax = s.max_batch;
-  a.group = 8;
+  // (probe-sign, M-tile) panels walked together, each W panel crossing HBM
+  // once per group: 12 where an A panel (256 rows x the launch's K, bf16) is
+  // 4 MB or more (K >= 8192: the 270M layer-1 and 1.1B launches, measured
+  // ~1% faster than 8), else 8 (smaller panels measured ~1% slower with more)
+  a.group = (a.nk - a.kbeg) * 64 >= 8192 ? 12 : 8;
   a.seed = seed;
   a.probe0 = probe0;
   a.eps = eps;
@@ -1289,7 +1293,11 @@ cudaError_t launch_loss_tc(const zo_ctx* ctx, const int32_t* targets, int t, int
   a.nk = H / 64;
   a.B = B;
   a.Bmax = s.max_batch;
-  a.group = 8;
+  // (probe-sign, M-tile) panels walked together, each W panel crossing HBM
+  // once per group: 12 where an A panel (256 rows x the launch's K, bf16) is
+  // 4 MB or more (K >= 8192: the 270M layer-1 and 1.1B launches, measured
+  // ~1% faster than 8), else 8 (smaller panels measured ~1% slower with more)
+  a.group = (a.nk - a.kbeg) * 64 >= 8192 ? 12 : 8;
   a.seed = seed;
   a.probe0 = probe0;
   a.eps = eps;
