@@ -312,13 +312,16 @@ def roofline_for(cfg, kinds, clocks, pk, steps, n_rank):
 class OracleSampler:
     """The C++ fp64 oracle (as it stands) on bounded samples of one CD-RGE step
     of `cfg`, on this host's cores.  A sample is one probe (both signs) over
-    R2 = min(B, 8) batch rows plus the update of a contiguous run of m
+    R2 = min(B, 16) batch rows plus the update of a contiguous run of m
     parameters with all n_pert probes.  The oracle's time for one probe grows
     linearly in the rows it evaluates, t(r) = t(1) + (r - 1) s, with an
     intercept that does not shrink with rows (it rebuilds every perturbed
     weight at every step), so one probe at 1 row and at R2 rows fix the line,
     and a full step is extrapolated as
-        t_step = n_pert t(B) + t_update(m) d_pad / m."""
+        t_step = n_pert t(B) + t_update(m) d_pad / m.
+    t(1) is the faster of two timings after an untimed first call (thread
+    start-up and first touches would otherwise inflate the intercept and
+    flatten the line)."""
 
     def __init__(self, cfg, rank=0):
         from oracle import native
@@ -331,14 +334,17 @@ class OracleSampler:
         self.d_pad = int(self.theta.size)
         self.m = min(self.d_pad, 1 << 22)
         self.coef = np.random.default_rng(0).standard_normal(cfg.n_pert) * 1e-3
-        self.R2 = min(cfg.batch, 8)
+        self.R2 = min(cfg.batch, 16)
         self.rows = np.arange(self.R2)
         self.t1 = None
         if cfg.batch > 1:
-            t0 = time.perf_counter()
-            self.N.probe_row_losses(self.theta, self.spec, W.step_seed(0), [0], cfg.eps,
-                                    self.tok, self.tgt, rows=[0])
-            self.t1 = time.perf_counter() - t0       # one probe, both signs, one row
+            ts = []
+            for rep in range(3):                     # one probe, both signs, one row
+                t0 = time.perf_counter()
+                self.N.probe_row_losses(self.theta, self.spec, W.step_seed(rep), [0], cfg.eps,
+                                        self.tok, self.tgt, rows=[0])
+                ts.append(time.perf_counter() - t0)
+            self.t1 = min(ts[1:])
 
     def sample(self, k):
         """One timed sample with probe k mod n_pert; returns (t_forward, t_update)."""
